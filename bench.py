@@ -1,0 +1,387 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE decode hot path on B200 (one JSON line on rank 0).
+
+Workload (default): the 30-layer stack of the Gemma-like MoE layer (hidden
+2816, 128 routed experts, top-8, expert intermediate 704, shared intermediate
+2112, 4-bit group-64 experts, int8 router, per-expert router bias N(0, 1.5)),
+decoding 256 consecutive tokens at batch 1 with an fp16 residual stream and
+RMSNorm between layers; all experts resident in HBM (13.2 GB).  One step is
+the decode of all 256 tokens through the 30 layers.  Inputs are synthetic and
+seeded; the weights are larger than L2 and each token touches ~1.1 GB.
+
+Multi-GPU: the path does not shard (one decode stream per GPU); --gpus N runs
+N independent replicas, timed as the max over ranks.
+
+--impl reference times the CPU oracle on the host cores on a bounded sample
+of the same workload (one token-layer per step) and reports the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE decode tokens/s per layer-stack; achieved HBM GB/s vs B200 peak (1 GPU)"
+UNIT = "tokens/s"
+N_LAYERS = 30
+N_TOKENS = 256
+SEED = 0
+BIAS_STD = 1.5
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--layers", type=int, default=N_LAYERS)
+    p.add_argument("--tokens", type=int, default=N_TOKENS)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=15.0)
+    return p.parse_args()
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        self.proc = None
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        sel = str(device_index)
+        try:
+            pr = torch.cuda.get_device_properties(device_index)
+            sel = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+        except Exception:
+            pass
+        self.cmd = ["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                    "--format=csv,noheader,nounits", "-lms", "200"]
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        with open(self.tmp.name) as f:
+            for line in f:
+                parts = [v.strip() for v in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.tmp.name)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        reasons = set()
+        for r in rows:
+            for name, v in zip(self.NAMES, r[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------ workload ----
+def build_stack(device, n_layers):
+    from bit_quantized_expert_int8_b200 import synth
+    from bit_quantized_expert_int8_b200.config import LAYER
+    return [synth.layer_weights(LAYER, SEED, l, device, bias_std=BIAS_STD)
+            for l in range(n_layers)]
+
+
+def kernel_launches_per_token(n_layers):
+    # per token: load + store; per layer: rmsnorm, router, pairs, gate/up,
+    # down, combine
+    return 2 + 6 * n_layers
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from bit_quantized_expert_int8_b200 import moeq4, synth
+    from bit_quantized_expert_int8_b200.config import LAYER
+
+    rank, local_rank, world = env_rank()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=dev)
+    moeq4.load()
+    cfg = LAYER
+    L, T = args.layers, args.tokens
+    layers = build_stack(dev, L)
+    objs = [moeq4.Layer.from_dict(d) for d in layers]
+    h0 = synth.tokens(T, cfg.H, SEED + 1 + rank, dev)
+    h = h0.clone()
+    y_last = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
+    ctx = moeq4.Context(cfg, 1)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        h.copy_(h0)
+        moeq4.moe_stack_decode(ctx, objs, h, T, y_last)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    value = world * T / (ms_max / 1000.0)
+
+    # ---- end to end through the C ABI with host buffers
+    h_host = h0.cpu().pin_memory()
+    h_back = torch.empty_like(h_host).pin_memory()
+
+    def step_e2e():
+        h.copy_(h_host, non_blocking=True)
+        moeq4.moe_stack_decode(ctx, objs, h, T, y_last)
+        h_back.copy_(h, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step_e2e()
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step_e2e()
+    e1.record(stream)
+    barrier()
+    ms_e2e = e0.elapsed_time(e1) / args.steps
+    t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_value = world * T / (float(t.item()) / 1000.0)
+
+    # ---- dominant kernel: the grouped expert FFN of one token-layer
+    roof = roofline(ctx, layers, cfg, dev, stream)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(layers, cfg, args.cpu_seconds, h0)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic (seeded; N(0,0.02) weights quantised to "
+                                     "4-bit group-64 and int8 router; N(0,1) fp16 tokens)",
+            "config": {"workload": f"stack{L}x{T}: {L}-layer MoE stack, {T} tokens decoded "
+                                   "one after another at batch 1",
+                       "hidden": cfg.H, "experts": cfg.E, "top_k": cfg.k,
+                       "inter": cfg.I, "inter_shared": cfg.Is, "group": 64,
+                       "router_bias_std": BIAS_STD, "tokens_per_step": T, "layers": L,
+                       "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (13.2 GB resident weights; "
+                             "~1.1 GB touched per token)"},
+            "e2e": {"value": round(e2e_value, 3), "unit": UNIT,
+                    "h2d_bytes_per_step": T * cfg.H * 2, "d2h_bytes_per_step": T * cfg.H * 2},
+            "gpu_launches": kernel_launches_per_token(L) * T * args.steps,
+            "roofline": roof,
+            "clocks": clk,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def roofline(ctx, layers, cfg, dev, stream):
+    """Average duration of one grouped-FFN launch (shared + 8 routed experts
+    of one token) over graph replays that rotate through all layers, so no
+    weight is L2-resident; algorithmic bytes = the 9 experts' blobs."""
+    import torch
+
+    from bit_quantized_expert_int8_b200 import moeq4, synth
+    hbm, kind = peaks()
+    n = len(layers)
+    nb = synth.blob_bytes(cfg.H, cfg.I)
+    x = synth.tokens(1, cfg.H, SEED + 77, dev)
+    idx = torch.empty((1, cfg.k), dtype=torch.int32, device=dev)
+    w = torch.empty((1, cfg.k), dtype=torch.float32, device=dev)
+    pairs = []
+    for d in layers:
+        moeq4.moe_router_topk(ctx, d["router_w"], d["router_scale"], d["router_bias"], x, 1,
+                              idx, w)
+        sel = idx[0].tolist()
+        base = d["experts"].data_ptr()
+        ent = [(d["shared"].data_ptr(), cfg.Is, 0)] + [(base + e * nb, cfg.I, 0) for e in sel]
+        pairs.append(moeq4.make_pairs(ent, dev))
+    y = torch.empty((cfg.k + 1, cfg.H), dtype=torch.float32, device=dev)
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for p in pairs:                                       # warm up
+            moeq4.moe_expert_ffn_q4(ctx, p, cfg.k + 1, x, 1, y, stream=side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for p in pairs:
+                moeq4.moe_expert_ffn_q4(ctx, p, cfg.k + 1, x, 1, y, stream=side)
+        reps = 20
+        for _ in range(3):
+            g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(side)
+        for _ in range(reps):
+            g.replay()
+        e1.record(side)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1000.0 / (reps * n)
+    algo = 8 * nb + synth.blob_bytes(cfg.H, cfg.Is)
+    achieved = algo / (us * 1e-6) / 1e9
+    return {"bound": "hbm", "kernel": "moe_expert_ffn_q4 (9 experts, one token)",
+            "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "peak_kind": f"{kind} (hbm_gbs)",
+            "algorithmic_bytes_per_launch": algo, "us_per_launch": round(us, 3),
+            "traffic": None}
+
+
+def cpu_baseline(layers, cfg, seconds, h0=None, n_sample_layers=2):
+    """The CPU oracle as it stands on the host cores: full MoE layers of this
+    workload, one token at a time, for about `seconds`; tokens/s of the whole
+    stack = 1 / (layers * mean seconds per token-layer)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from bit_quantized_expert_int8_b200 import synth
+    cores = oracle.set_threads(0)
+    lns = []
+    for d in layers[:n_sample_layers]:
+        lns.append({k: (None if v is None else
+                        (v.cpu().view(torch.int16).numpy().view(np.uint16)
+                         if v.dtype == torch.float16 else v.cpu().numpy()))
+                    for k, v in d.items()})
+    x = synth.tokens(64, cfg.H, SEED + 5, "cpu").view(torch.int16).numpy().view(np.uint16)
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.moe_layer(cfg, lns[n % len(lns)], x[n % x.shape[0]])
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    per = el / n
+    return {"value": round(1.0 / (N_LAYERS * per), 5), "unit": UNIT, "cores": cores,
+            "kind": "oracle",
+            "sample": f"{n} token-layers of the stack workload (layers 0-{len(lns) - 1}), "
+                      f"{per * 1e3:.1f} ms each; tokens/s = 1/({N_LAYERS} x that)"}
+
+
+def run_reference(args):
+    rank, _, world = env_rank()
+    if rank != 0:
+        return
+    import torch
+
+    import oracle
+    from bit_quantized_expert_int8_b200.config import LAYER
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    layers = build_stack(dev, 2)
+    cfg = LAYER
+    per_step = []
+    cores = oracle.set_threads(0)
+    import numpy as np
+
+    from bit_quantized_expert_int8_b200 import synth
+    lns = [{k: (None if v is None else
+                (v.cpu().view(torch.int16).numpy().view(np.uint16)
+                 if v.dtype == torch.float16 else v.cpu().numpy()))
+            for k, v in d.items()} for d in layers]
+    x = synth.tokens(64, cfg.H, SEED + 5, "cpu").view(torch.int16).numpy().view(np.uint16)
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.moe_layer(cfg, lns[i % 2], x[i % 64])
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            per_step.append(dt)
+    per = sum(per_step) / len(per_step)
+    value = 1.0 / (N_LAYERS * per)
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(per * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (same recipe as ours)",
+            "config": {"workload": f"stack{args.layers}x{args.tokens} (one token-layer "
+                                   "sampled per step)", "hidden": cfg.H, "experts": cfg.E,
+                       "top_k": cfg.k, "inter": cfg.I, "inter_shared": cfg.Is},
+            "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"{args.steps} token-layers (layers 0-1), "
+                                       f"{per * 1e3:.1f} ms each"},
+            "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,461 @@
+// moeq4_api.cu -- the C ABI of libmoeq4.so (declared in include/moeq4.h).
+//
+// Host side: argument checks, workspace, stream/event plumbing and launches.
+// Every arithmetic step of the path runs in the kernels included below.
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "ffn_simple.cuh"
+#include "misc.cuh"
+#include "router.cuh"
+
+using namespace moeq4;
+
+// ------------------------------------------------------------ errors --
+static thread_local std::string g_err;
+
+static int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+#define CK(call)                                                                   \
+    do {                                                                           \
+        cudaError_t e_ = (call);                                                   \
+        if (e_ != cudaSuccess)                                                     \
+            return fail(MOE_ERR_CUDA, "%s: %s (%s:%d)", #call, cudaGetErrorString(e_), \
+                        __FILE__, __LINE__);                                       \
+    } while (0)
+
+#define CKL() CK(cudaGetLastError())
+
+#define TRY(expr)                 \
+    do {                          \
+        int rc_ = (expr);         \
+        if (rc_ != MOE_OK) return rc_; \
+    } while (0)
+
+static inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// ------------------------------------------------------------ context --
+struct StackKey {
+    std::vector<MoeLayer> layers;
+    moe_half* h = nullptr;
+    float* y_last = nullptr;
+};
+
+struct moe_ctx {
+    MoeConfig cfg{};
+    int maxT = 0;
+    int device = 0;
+    int maxI = 0;
+    // device workspace (one allocation)
+    uint8_t* ws = nullptr;
+    double* logits = nullptr;
+    int* router_done = nullptr;
+    int32_t* idx = nullptr;
+    float* w = nullptr;
+    MoeFfnPair* pairs = nullptr;
+    float* h_ws = nullptr;
+    float* y_pairs = nullptr;
+    __half* x_norm = nullptr;
+    int32_t* slot_of = nullptr;
+    int* cursor = nullptr;
+    __half* h_cur = nullptr;
+    float* y_cur = nullptr;
+    // mapped pinned host memory for the streaming miss list
+    int32_t* miss_host = nullptr;    // [maxT*k*2 + 4]; last words hold n_miss
+    int32_t* miss_dev = nullptr;
+    int32_t* n_miss_host = nullptr;
+    int32_t* n_miss_dev = nullptr;
+    cudaEvent_t ev_lookup = nullptr, ev_copy = nullptr;
+    cudaStream_t cap_stream = nullptr;
+    // stack graph
+    cudaGraphExec_t stack_exec = nullptr;
+    StackKey stack_key;
+    // host-side fault injection (tests): fail the Nth blob copy before issue
+    long fail_copy_at = -1;
+    long copies_seen = 0;
+};
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+static int check_cfg(const MoeConfig* c) {
+    if (!c) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+    if (c->hidden <= 0 || c->hidden % MOE_GROUP || c->inter <= 0 || c->inter % MOE_GROUP ||
+        c->inter_shared <= 0 || c->inter_shared % MOE_GROUP)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                    "hidden/inter/inter_shared must be positive multiples of 64 (%d, %d, %d)",
+                    c->hidden, c->inter, c->inter_shared);
+    if (c->hidden > 16384 || c->inter > 16384 || c->inter_shared > 16384)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "hidden/inter above 16384");
+    if (c->top_k < 1 || c->top_k > MOE_MAX_TOPK || c->n_experts < c->top_k ||
+        c->n_experts > MOE_MAX_EXPERTS)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "need 1 <= top_k <= 8, top_k <= n_experts <= 256");
+    if (c->n_slots <= c->top_k || c->n_slots > MOE_MAX_SLOTS)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "need top_k < n_slots <= 32");
+    if ((c->renorm != 0 && c->renorm != 1) || (c->gelu != MOE_GELU_TANH && c->gelu != MOE_GELU_ERF))
+        return fail(MOE_ERR_INVALID_ARG, "renorm must be 0/1 and gelu a MOE_GELU_* value");
+    if (!(c->rms_eps >= 0.0)) return fail(MOE_ERR_INVALID_ARG, "rms_eps must be >= 0");
+    return MOE_OK;
+}
+
+extern "C" const char* moe_last_error(void) { return g_err.c_str(); }
+
+extern "C" size_t moe_blob_bytes(int hidden, int inter) {
+    if (hidden <= 0 || inter <= 0 || hidden % MOE_GROUP || inter % MOE_GROUP) return 0;
+    return BlobLayout(hidden, inter).bytes;
+}
+
+extern "C" int moe_ctx_destroy(moe_ctx* c) {
+    if (!c) return MOE_OK;
+    cudaSetDevice(c->device);
+    cudaDeviceSynchronize();
+    if (c->stack_exec) cudaGraphExecDestroy(c->stack_exec);
+    if (c->ev_lookup) cudaEventDestroy(c->ev_lookup);
+    if (c->ev_copy) cudaEventDestroy(c->ev_copy);
+    if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
+    if (c->miss_host) cudaFreeHost(c->miss_host);
+    if (c->ws) cudaFree(c->ws);
+    delete c;
+    return MOE_OK;
+}
+
+extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** out) {
+    if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    TRY(check_cfg(cfg));
+    if (max_tokens < 1 || max_tokens > 65535)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "max_tokens must be 1..65535");
+    moe_ctx* c = new moe_ctx();
+    c->cfg = *cfg;
+    c->maxT = max_tokens;
+    c->maxI = cfg->inter > cfg->inter_shared ? cfg->inter : cfg->inter_shared;
+    cudaGetDevice(&c->device);
+    const size_t T = max_tokens, E = cfg->n_experts, k = cfg->top_k, H = cfg->hidden;
+    const size_t P = T * (k + 1);
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+    size_t o_logits = take(T * E * sizeof(double));
+    size_t o_done = take(T * sizeof(int));
+    size_t o_idx = take(T * k * sizeof(int32_t));
+    size_t o_w = take(T * k * sizeof(float));
+    size_t o_pairs = take(P * sizeof(MoeFfnPair));
+    size_t o_h = take(P * (size_t)c->maxI * sizeof(float));
+    size_t o_y = take(P * H * sizeof(float));
+    size_t o_xn = take(T * H * sizeof(__half));
+    size_t o_slot = take(T * k * sizeof(int32_t));
+    size_t o_cur = take(sizeof(int));
+    size_t o_hcur = take(H * sizeof(__half));
+    size_t o_ycur = take(H * sizeof(float));
+    int rc = MOE_OK;
+    cudaError_t e = cudaMalloc(&c->ws, off);
+    if (e == cudaSuccess) e = cudaMemset(c->ws, 0, off);
+    if (e == cudaSuccess) {
+        c->logits = (double*)(c->ws + o_logits);
+        c->router_done = (int*)(c->ws + o_done);
+        c->idx = (int32_t*)(c->ws + o_idx);
+        c->w = (float*)(c->ws + o_w);
+        c->pairs = (MoeFfnPair*)(c->ws + o_pairs);
+        c->h_ws = (float*)(c->ws + o_h);
+        c->y_pairs = (float*)(c->ws + o_y);
+        c->x_norm = (__half*)(c->ws + o_xn);
+        c->slot_of = (int32_t*)(c->ws + o_slot);
+        c->cursor = (int*)(c->ws + o_cur);
+        c->h_cur = (__half*)(c->ws + o_hcur);
+        c->y_cur = (float*)(c->ws + o_ycur);
+        size_t nm = T * k * 2 + 4;
+        e = cudaHostAlloc((void**)&c->miss_host, nm * sizeof(int32_t), cudaHostAllocMapped);
+    }
+    if (e == cudaSuccess) e = cudaHostGetDevicePointer((void**)&c->miss_dev, c->miss_host, 0);
+    if (e == cudaSuccess) {
+        c->n_miss_host = c->miss_host + T * k * 2;
+        c->n_miss_dev = c->miss_dev + T * k * 2;
+        e = cudaEventCreateWithFlags(&c->ev_lookup, cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_copy, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking);
+    const int smem_router = (int)(H * sizeof(long long));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_router);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_ffn_gateup_simple, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(H * sizeof(float)));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_ffn_down_simple, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(c->maxI * sizeof(float)));
+    if (e != cudaSuccess) {
+        rc = fail(MOE_ERR_CUDA, "moe_ctx_create: %s", cudaGetErrorString(e));
+        moe_ctx_destroy(c);
+        return rc;
+    }
+    if (const char* f = getenv("MOEQ4_FAIL_COPY_AT")) c->fail_copy_at = atol(f);
+    *out = c;
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------- launches --
+static int launch_router(moe_ctx* c, const int8_t* Wr, const moe_half* sc, const float* bias,
+                         const __half* x, int T, int32_t* idx, float* w, double* logits,
+                         cudaStream_t s) {
+    const MoeConfig& g = c->cfg;
+    dim3 grid((g.n_experts + kRouterWarps - 1) / kRouterWarps, T);
+    k_router<<<grid, 256, g.hidden * sizeof(long long), s>>>(
+        Wr, reinterpret_cast<const __half*>(sc), bias, x, g.n_experts, g.hidden, g.top_k,
+        g.renorm, logits ? logits : c->logits, c->router_done, idx, w);
+    CKL();
+    return MOE_OK;
+}
+
+static int launch_ffn(moe_ctx* c, const MoeFfnPair* pairs, int n, const __half* x, int T,
+                      float* h_ws, float* y, cudaStream_t s) {
+    const MoeConfig& g = c->cfg;
+    dim3 g1((c->maxI + 7) / 8, n);
+    k_ffn_gateup_simple<<<g1, 256, g.hidden * sizeof(float), s>>>(
+        pairs, x, T, g.hidden, g.inter, g.inter_shared, g.gelu, h_ws, c->maxI);
+    CKL();
+    dim3 g2(g.hidden / 8, n);
+    k_ffn_down_simple<<<g2, 256, c->maxI * sizeof(float), s>>>(pairs, h_ws, c->maxI, g.hidden,
+                                                               g.inter, g.inter_shared, y);
+    CKL();
+    return MOE_OK;
+}
+
+static int launch_combine(moe_ctx* c, const float* y_routed, const float* y_shared,
+                          const float* w, int T, float* y, __half* residual, cudaStream_t s) {
+    const MoeConfig& g = c->cfg;
+    dim3 grid((g.hidden + 255) / 256, T);
+    k_combine<<<grid, 256, 0, s>>>(y_routed, (size_t)g.top_k * g.hidden, y_shared, g.hidden, w,
+                                   g.top_k, g.hidden, y, residual);
+    CKL();
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------- exports --
+extern "C" int moe_router_topk(moe_ctx* c, const int8_t* Wr, const moe_half* row_scale,
+                               const float* bias, const moe_half* x, int T, int32_t* topk_idx,
+                               float* topk_w, double* logits, moe_stream_t stream) {
+    if (!c || !Wr || !row_scale || !x || !topk_idx || !topk_w)
+        return fail(MOE_ERR_INVALID_ARG, "moe_router_topk: NULL argument");
+    if (T < 1 || T > c->maxT) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T=%d outside 1..%d", T, c->maxT);
+    if (!aligned16(Wr) || !aligned16(row_scale) || !aligned16(x) || !aligned16(topk_idx) ||
+        !aligned16(topk_w) || (bias && !aligned16(bias)) || (logits && !aligned16(logits)))
+        return fail(MOE_ERR_ALIGNMENT, "moe_router_topk: pointers must be 16-byte aligned");
+    return launch_router(c, Wr, row_scale, bias, reinterpret_cast<const __half*>(x), T, topk_idx,
+                         topk_w, logits, stream);
+}
+
+extern "C" int moe_expert_ffn_q4(moe_ctx* c, const MoeFfnPair* pairs, int n_pairs,
+                                 const moe_half* x, int T, float* y, moe_stream_t stream) {
+    if (!c || !pairs || !x || !y) return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn_q4: NULL argument");
+    if (n_pairs < 1 || n_pairs > c->maxT * (c->cfg.top_k + 1))
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n_pairs=%d outside 1..%d", n_pairs,
+                    c->maxT * (c->cfg.top_k + 1));
+    if (T < 1) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T must be >= 1");
+    if (!aligned16(pairs) || !aligned16(x) || !aligned16(y))
+        return fail(MOE_ERR_ALIGNMENT, "moe_expert_ffn_q4: pointers must be 16-byte aligned");
+    return launch_ffn(c, pairs, n_pairs, reinterpret_cast<const __half*>(x), T, c->h_ws, y,
+                      stream);
+}
+
+extern "C" int moe_combine(moe_ctx* c, const float* y_routed, const float* y_shared,
+                           const float* topk_w, int T, float* y_out, moe_half* residual,
+                           moe_stream_t stream) {
+    if (!c || !y_routed || !y_shared || !topk_w || !y_out)
+        return fail(MOE_ERR_INVALID_ARG, "moe_combine: NULL argument");
+    if (T < 1 || T > 65535) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T=%d outside 1..65535", T);
+    if (!aligned16(y_routed) || !aligned16(y_shared) || !aligned16(topk_w) || !aligned16(y_out) ||
+        (residual && !aligned16(residual)))
+        return fail(MOE_ERR_ALIGNMENT, "moe_combine: pointers must be 16-byte aligned");
+    return launch_combine(c, y_routed, y_shared, topk_w, T, y_out,
+                          reinterpret_cast<__half*>(residual), stream);
+}
+
+extern "C" int moe_lfu_init(moe_ctx* c, MoeLfuTable* table, int n_slots, moe_stream_t stream) {
+    if (!c || !table) return fail(MOE_ERR_INVALID_ARG, "moe_lfu_init: NULL argument");
+    if (n_slots <= c->cfg.top_k || n_slots > MOE_MAX_SLOTS)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "need top_k < n_slots <= 32 (got %d)", n_slots);
+    if (!aligned16(table)) return fail(MOE_ERR_ALIGNMENT, "table must be 16-byte aligned");
+    k_lfu_init<<<1, 32, 0, stream>>>(table, n_slots);
+    CKL();
+    return MOE_OK;
+}
+
+extern "C" int moe_cache_lookup_lfu(moe_ctx* c, MoeLfuTable* table, const int32_t* topk_idx,
+                                    int T, int32_t* slot_of, int32_t* miss_list, int32_t* n_miss,
+                                    moe_stream_t stream) {
+    if (!c || !table || !topk_idx || !slot_of || !miss_list || !n_miss)
+        return fail(MOE_ERR_INVALID_ARG, "moe_cache_lookup_lfu: NULL argument");
+    if (T < 1 || T > 65535) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T=%d outside 1..65535", T);
+    if (!aligned16(table) || !aligned16(topk_idx) || !aligned16(slot_of) || !aligned16(miss_list))
+        return fail(MOE_ERR_ALIGNMENT, "moe_cache_lookup_lfu: pointers must be 16-byte aligned");
+    k_lfu_lookup<<<1, 32, 0, stream>>>(table, topk_idx, T, c->cfg.top_k, slot_of, miss_list, n_miss);
+    CKL();
+    return MOE_OK;
+}
+
+// Resident layer body on one stream (also used inside the stack capture).
+static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const MoeLayerOut* o,
+                          int flags, cudaStream_t s) {
+    const MoeConfig& g = c->cfg;
+    const int k = g.top_k, H = g.hidden;
+    const __half* xin = x;
+    __half* xn = o->x_norm ? reinterpret_cast<__half*>(o->x_norm) : c->x_norm;
+    if (flags & MOE_PRENORM) {
+        k_rmsnorm<<<T, 256, 0, s>>>(x, xn, H, g.rms_eps);
+        CKL();
+        xin = xn;
+    }
+    int32_t* idx = o->topk_idx ? o->topk_idx : c->idx;
+    float* w = o->topk_w ? o->topk_w : c->w;
+    TRY(launch_router(c, L->router_w, L->router_scale, L->router_bias, xin, T, idx, w, nullptr, s));
+    const size_t stride = BlobLayout(H, g.inter).bytes;
+    const int P = T * (k + 1);
+    k_build_pairs<<<(P + 127) / 128, 128, 0, s>>>(L->shared_blob, g.inter_shared,
+                                                  static_cast<const uint8_t*>(L->experts), stride,
+                                                  idx, g.inter, T, k, c->pairs);
+    CKL();
+    TRY(launch_ffn(c, c->pairs, P, xin, T, c->h_ws, c->y_pairs, s));
+    TRY(launch_combine(c, c->y_pairs + (size_t)T * H, c->y_pairs, w, T, o->y,
+                       (flags & MOE_PRENORM) ? x : nullptr, s));
+    return MOE_OK;
+}
+
+static int layer_streaming(moe_ctx* c, const MoeLayer* L, __half* x, const MoeLayerOut* o,
+                           int flags, cudaStream_t s, cudaStream_t cs) {
+    const MoeConfig& g = c->cfg;
+    const int k = g.top_k, H = g.hidden, T = 1;
+    const __half* xin = x;
+    __half* xn = o->x_norm ? reinterpret_cast<__half*>(o->x_norm) : c->x_norm;
+    if (flags & MOE_PRENORM) {
+        k_rmsnorm<<<T, 256, 0, s>>>(x, xn, H, g.rms_eps);
+        CKL();
+        xin = xn;
+    }
+    int32_t* idx = o->topk_idx ? o->topk_idx : c->idx;
+    float* w = o->topk_w ? o->topk_w : c->w;
+    int32_t* slot_of = o->slot_of ? o->slot_of : c->slot_of;
+    TRY(launch_router(c, L->router_w, L->router_scale, L->router_bias, xin, T, idx, w, nullptr, s));
+    k_lfu_lookup<<<1, 32, 0, s>>>(L->lfu, idx, T, k, slot_of, c->miss_dev, c->n_miss_dev);
+    CKL();
+    CK(cudaEventRecord(c->ev_lookup, s));
+    const size_t stride = BlobLayout(H, g.inter).bytes;
+    k_build_pairs<<<1, 128, 0, s>>>(L->shared_blob, g.inter_shared,
+                                    static_cast<const uint8_t*>(L->slots), stride, slot_of,
+                                    g.inter, T, k, c->pairs);
+    CKL();
+    // shared branch computes while the misses are fetched
+    TRY(launch_ffn(c, c->pairs, T, xin, T, c->h_ws, c->y_pairs, s));
+    CK(cudaEventSynchronize(c->ev_lookup));
+    const int nm = *(volatile int32_t*)c->n_miss_host;
+    if (nm < 0) return fail(MOE_ERR_CACHE_STATE, "LFU table is invalid (an earlier fill failed)");
+    const uint8_t* store = static_cast<const uint8_t*>(L->host_store);
+    uint8_t* slots = static_cast<uint8_t*>(L->slots);
+    for (int i = 0; i < nm; i++) {
+        const int e = c->miss_host[2 * i], slot = c->miss_host[2 * i + 1];
+        cudaError_t err = cudaSuccess;
+        if (c->fail_copy_at >= 0 && c->copies_seen == c->fail_copy_at) err = cudaErrorInvalidValue;
+        c->copies_seen++;
+        if (err == cudaSuccess)
+            err = cudaMemcpyAsync(slots + (size_t)slot * stride, store + (size_t)e * stride, stride,
+                                  cudaMemcpyHostToDevice, cs);
+        if (err != cudaSuccess) {
+            k_lfu_invalidate<<<1, 1, 0, s>>>(L->lfu);
+            return fail(MOE_ERR_CACHE_STATE, "fill of expert %d into slot %d failed: %s; table "
+                        "marked invalid", e, slot, cudaGetErrorString(err));
+        }
+    }
+    CK(cudaEventRecord(c->ev_copy, cs));
+    CK(cudaStreamWaitEvent(s, c->ev_copy, 0));
+    TRY(launch_ffn(c, c->pairs + T, T * k, xin, T, c->h_ws + (size_t)T * c->maxI,
+                   c->y_pairs + (size_t)T * H, s));
+    TRY(launch_combine(c, c->y_pairs + (size_t)T * H, c->y_pairs, w, T, o->y,
+                       (flags & MOE_PRENORM) ? x : nullptr, s));
+    return MOE_OK;
+}
+
+extern "C" int moe_layer_decode(moe_ctx* c, const MoeLayer* L, moe_half* x, int T,
+                                const MoeLayerOut* o, int flags, moe_stream_t main,
+                                moe_stream_t copy) {
+    if (!c || !L || !x || !o || !o->y) return fail(MOE_ERR_INVALID_ARG, "moe_layer_decode: NULL argument");
+    if (flags & ~MOE_PRENORM) return fail(MOE_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+    if (T < 1 || T > c->maxT) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T=%d outside 1..%d", T, c->maxT);
+    if (!L->router_w || !L->router_scale || !L->shared_blob)
+        return fail(MOE_ERR_INVALID_ARG, "layer needs router_w, router_scale and shared_blob");
+    const void* ptrs[] = {L->router_w, L->router_scale, L->shared_blob, x, o->y};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return fail(MOE_ERR_ALIGNMENT, "moe_layer_decode: pointers must be 16-byte aligned");
+    if ((L->router_bias && !aligned16(L->router_bias)) || (o->topk_idx && !aligned16(o->topk_idx)) ||
+        (o->topk_w && !aligned16(o->topk_w)) || (o->slot_of && !aligned16(o->slot_of)) ||
+        (o->x_norm && !aligned16(o->x_norm)))
+        return fail(MOE_ERR_ALIGNMENT, "moe_layer_decode: pointers must be 16-byte aligned");
+    if (L->experts) {
+        if (!aligned16(L->experts)) return fail(MOE_ERR_ALIGNMENT, "experts must be 16-byte aligned");
+        return layer_resident(c, L, reinterpret_cast<__half*>(x), T, o, flags, main);
+    }
+    if (!L->host_store || !L->slots || !L->lfu || !copy)
+        return fail(MOE_ERR_INVALID_ARG, "streaming mode needs host_store, slots, lfu and a copy stream");
+    if (T != 1) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "streaming mode decodes one token per call");
+    if (!aligned16(L->slots) || !aligned16(L->lfu) || !aligned16(L->host_store))
+        return fail(MOE_ERR_ALIGNMENT, "moe_layer_decode: pointers must be 16-byte aligned");
+    return layer_streaming(c, L, reinterpret_cast<__half*>(x), o, flags, main, copy);
+}
+
+static bool same_key(const StackKey& k, const MoeLayer* layers, int n, moe_half* h, float* y) {
+    if ((int)k.layers.size() != n || k.h != h || k.y_last != y) return false;
+    return memcmp(k.layers.data(), layers, sizeof(MoeLayer) * n) == 0;
+}
+
+extern "C" int moe_stack_decode(moe_ctx* c, const MoeLayer* layers, int n_layers, moe_half* h,
+                                int T, float* y_last, moe_stream_t stream) {
+    if (!c || !layers || !h) return fail(MOE_ERR_INVALID_ARG, "moe_stack_decode: NULL argument");
+    if (n_layers < 1 || T < 1) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n_layers and T must be >= 1");
+    if (!aligned16(h) || (y_last && !aligned16(y_last)))
+        return fail(MOE_ERR_ALIGNMENT, "moe_stack_decode: pointers must be 16-byte aligned");
+    for (int l = 0; l < n_layers; l++) {
+        const MoeLayer& L = layers[l];
+        if (!L.router_w || !L.router_scale || !L.shared_blob || !L.experts)
+            return fail(MOE_ERR_INVALID_ARG, "layer %d is not a resident layer", l);
+        if (!aligned16(L.router_w) || !aligned16(L.router_scale) || !aligned16(L.shared_blob) ||
+            !aligned16(L.experts) || (L.router_bias && !aligned16(L.router_bias)))
+            return fail(MOE_ERR_ALIGNMENT, "layer %d: pointers must be 16-byte aligned", l);
+    }
+    const int H = c->cfg.hidden;
+    if (!c->stack_exec || !same_key(c->stack_key, layers, n_layers, h, y_last)) {
+        if (c->stack_exec) { cudaGraphExecDestroy(c->stack_exec); c->stack_exec = nullptr; }
+        cudaStream_t cs = c->cap_stream;
+        CK(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
+        int rc = MOE_OK;
+        k_copy_half_row<<<1, 256, 0, cs>>>(reinterpret_cast<__half*>(h), c->h_cur, c->cursor, H, 1);
+        MoeLayerOut o{};
+        o.y = c->y_cur;
+        for (int l = 0; l < n_layers && rc == MOE_OK; l++)
+            rc = layer_resident(c, &layers[l], c->h_cur, 1, &o, MOE_PRENORM, cs);
+        if (rc == MOE_OK)
+            k_store_token<<<1, 256, 0, cs>>>(c->h_cur, c->y_cur, reinterpret_cast<__half*>(h), y_last,
+                                             c->cursor, H);
+        cudaGraph_t graph = nullptr;
+        cudaError_t e = cudaStreamEndCapture(cs, &graph);
+        if (rc != MOE_OK) { if (graph) cudaGraphDestroy(graph); return rc; }
+        if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "stack capture: %s", cudaGetErrorString(e));
+        e = cudaGraphInstantiate(&c->stack_exec, graph, 0);
+        cudaGraphDestroy(graph);
+        if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "stack instantiate: %s", cudaGetErrorString(e));
+        c->stack_key.layers.assign(layers, layers + n_layers);
+        c->stack_key.h = h;
+        c->stack_key.y_last = y_last;
+    }
+    CK(cudaMemsetAsync(c->cursor, 0, sizeof(int), stream));
+    for (int t = 0; t < T; t++) CK(cudaGraphLaunch(c->stack_exec, stream));
+    return MOE_OK;
+}

@@ -1,0 +1,230 @@
+"""ctypes binding of libmoeq4.so: the C ABI of include/moeq4.h, same names.
+
+Argument marshalling only: torch tensors are passed as raw device pointers and
+streams as their CUDA handles; every step of the path runs in the library's
+kernels.  There is no fallback: if the shared library is missing or cannot be
+loaded, ``load()`` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .config import MoeConfig
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoeq4.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_ALIGNMENT = -2
+MOE_ERR_UNSUPPORTED_SHAPE = -3
+MOE_ERR_CUDA = -4
+MOE_ERR_TIMEOUT = -5
+MOE_ERR_CACHE_STATE = -6
+MOE_PRENORM = 1
+MOE_MAX_SLOTS = 32
+
+EXPORTS = ("moe_ctx_create", "moe_ctx_destroy", "moe_last_error", "moe_blob_bytes",
+           "moe_router_topk", "moe_expert_ffn_q4", "moe_combine", "moe_lfu_init",
+           "moe_cache_lookup_lfu", "moe_layer_decode", "moe_stack_decode")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"moeq4 error {code}: {msg}")
+        self.code = code
+
+
+class CMoeConfig(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("n_experts", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("inter", ctypes.c_int32),
+                ("inter_shared", ctypes.c_int32), ("n_slots", ctypes.c_int32),
+                ("renorm", ctypes.c_int32), ("gelu", ctypes.c_int32),
+                ("rms_eps", ctypes.c_double)]
+
+
+class CMoeLayer(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "router_w", "router_scale", "router_bias", "shared_blob", "experts",
+        "host_store", "slots", "lfu")]
+
+
+class CMoeLayerOut(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("y", "topk_idx", "topk_w", "slot_of", "x_norm")]
+
+
+class CMoeLfuTable(ctypes.Structure):
+    _fields_ = [("expert", ctypes.c_int32 * MOE_MAX_SLOTS),
+                ("count", ctypes.c_int64 * MOE_MAX_SLOTS),
+                ("seq", ctypes.c_int64 * MOE_MAX_SLOTS),
+                ("counter", ctypes.c_int64), ("hits", ctypes.c_int64),
+                ("misses", ctypes.c_int64), ("n_slots", ctypes.c_int32),
+                ("valid", ctypes.c_int32)]
+
+
+LFU_TABLE_BYTES = ctypes.sizeof(CMoeLfuTable)
+PAIR_BYTES = 16   # MoeFfnPair: blob pointer, int32 inter, int32 token
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libmoeq4.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with "
+                          "bit_quantized_expert_int8_b200.build.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i32 = ctypes.c_void_p, ctypes.c_int
+    sig = {
+        "moe_ctx_create": ([ctypes.POINTER(CMoeConfig), i32, ctypes.POINTER(P)], i32),
+        "moe_ctx_destroy": ([P], i32),
+        "moe_last_error": ([], ctypes.c_char_p),
+        "moe_blob_bytes": ([i32, i32], ctypes.c_size_t),
+        "moe_router_topk": ([P, P, P, P, P, i32, P, P, P, P], i32),
+        "moe_expert_ffn_q4": ([P, P, i32, P, i32, P, P], i32),
+        "moe_combine": ([P, P, P, P, i32, P, P, P], i32),
+        "moe_lfu_init": ([P, P, i32, P], i32),
+        "moe_cache_lookup_lfu": ([P, P, P, i32, P, P, P, P], i32),
+        "moe_layer_decode": ([P, ctypes.POINTER(CMoeLayer), P, i32,
+                              ctypes.POINTER(CMoeLayerOut), i32, P, P], i32),
+        "moe_stack_decode": ([P, P, i32, P, i32, P, P], i32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(rc: int):
+    if rc != MOE_OK:
+        raise MoeError(rc, load().moe_last_error().decode())
+
+
+def last_error() -> str:
+    return load().moe_last_error().decode()
+
+
+def blob_bytes(hidden: int, inter: int) -> int:
+    return int(load().moe_blob_bytes(hidden, inter))
+
+
+class Context:
+    """moe_ctx_create / moe_ctx_destroy."""
+
+    def __init__(self, cfg: MoeConfig, max_tokens: int = 1):
+        lib = load()
+        self.cfg = cfg
+        self.max_tokens = max_tokens
+        self._c = CMoeConfig(cfg.H, cfg.E, cfg.k, cfg.I, cfg.Is, cfg.S,
+                             cfg.renorm, cfg.gelu, cfg.rms_eps)
+        h = ctypes.c_void_p()
+        _check(lib.moe_ctx_create(ctypes.byref(self._c), max_tokens, ctypes.byref(h)))
+        self.handle = h.value
+
+    def close(self):
+        if self.handle:
+            load().moe_ctx_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def moe_router_topk(ctx, Wr, row_scale, bias, x, T, topk_idx, topk_w, logits=None, stream=None):
+    _check(load().moe_router_topk(ctx.handle, _ptr(Wr), _ptr(row_scale), _ptr(bias), _ptr(x), T,
+                                  _ptr(topk_idx), _ptr(topk_w), _ptr(logits), _stream(stream)))
+
+
+def make_pairs(entries, device="cuda"):
+    """Pack [(blob_ptr, inter, token), ...] into a device MoeFfnPair array."""
+    buf = torch.empty((len(entries), PAIR_BYTES), dtype=torch.uint8)
+    for i, (p, inter, tok) in enumerate(entries):
+        buf[i, :8] = torch.tensor([p], dtype=torch.int64).view(torch.uint8)
+        buf[i, 8:] = torch.tensor([inter, tok], dtype=torch.int32).view(torch.uint8)
+    return buf.to(device)
+
+
+def moe_expert_ffn_q4(ctx, pairs, n_pairs, x, T, y, stream=None):
+    _check(load().moe_expert_ffn_q4(ctx.handle, _ptr(pairs), n_pairs, _ptr(x), T, _ptr(y),
+                                    _stream(stream)))
+
+
+def moe_combine(ctx, y_routed, y_shared, topk_w, T, y_out, residual=None, stream=None):
+    _check(load().moe_combine(ctx.handle, _ptr(y_routed), _ptr(y_shared), _ptr(topk_w), T,
+                              _ptr(y_out), _ptr(residual), _stream(stream)))
+
+
+def new_lfu_table(device="cuda"):
+    """Device buffer large enough for one MoeLfuTable."""
+    return torch.zeros(LFU_TABLE_BYTES, dtype=torch.uint8, device=device)
+
+
+def read_lfu_table(table) -> CMoeLfuTable:
+    raw = table.cpu().numpy().tobytes()
+    return CMoeLfuTable.from_buffer_copy(raw)
+
+
+def moe_lfu_init(ctx, table, n_slots, stream=None):
+    _check(load().moe_lfu_init(ctx.handle, _ptr(table), n_slots, _stream(stream)))
+
+
+def moe_cache_lookup_lfu(ctx, table, topk_idx, T, slot_of, miss_list, n_miss, stream=None):
+    _check(load().moe_cache_lookup_lfu(ctx.handle, _ptr(table), _ptr(topk_idx), T,
+                                       _ptr(slot_of), _ptr(miss_list), _ptr(n_miss),
+                                       _stream(stream)))
+
+
+class Layer:
+    """A layer's buffers (torch tensors) as the C MoeLayer struct."""
+
+    def __init__(self, router_w, router_scale, router_bias=None, shared=None, experts=None,
+                 host_store=None, slots=None, lfu=None):
+        self.keep = (router_w, router_scale, router_bias, shared, experts, host_store, slots, lfu)
+        self.c = CMoeLayer(_ptr(router_w), _ptr(router_scale), _ptr(router_bias), _ptr(shared),
+                           _ptr(experts), _ptr(host_store), _ptr(slots), _ptr(lfu))
+
+    @classmethod
+    def from_dict(cls, d, **kw):
+        return cls(d["router_w"], d["router_scale"], d.get("router_bias"), d["shared"],
+                   d.get("experts"), **kw)
+
+
+def moe_layer_decode(ctx, layer: Layer, x, T, y, topk_idx=None, topk_w=None, slot_of=None,
+                     x_norm=None, flags=0, stream=None, copy_stream=None):
+    out = CMoeLayerOut(_ptr(y), _ptr(topk_idx), _ptr(topk_w), _ptr(slot_of), _ptr(x_norm))
+    cs = None if copy_stream is None else _stream(copy_stream)
+    _check(load().moe_layer_decode(ctx.handle, ctypes.byref(layer.c), _ptr(x), T,
+                                   ctypes.byref(out), flags, _stream(stream), cs))
+
+
+def moe_stack_decode(ctx, layers, h, T, y_last=None, stream=None):
+    arr = (CMoeLayer * len(layers))(*[l.c for l in layers])
+    _check(load().moe_stack_decode(ctx.handle, ctypes.cast(arr, ctypes.c_void_p), len(layers),
+                                   _ptr(h), T, _ptr(y_last), _stream(stream)))

@@ -1,0 +1,276 @@
+/*
+ * moeq4.h -- C ABI of libmoeq4.so, the B200 (sm_100a) MoE decode hot path.
+ *
+ * Per token and layer the path is: an 8-bit router picks the top 8 of 128
+ * routed experts; one shared expert and the 8 routed experts (4-bit affine
+ * weights) each run a gated FFN; the outputs are combined with the router
+ * weights; in streaming mode the missing experts are fetched into a 16-slot
+ * LFU cache per layer while the shared branch computes.
+ *
+ * Sources (web pages on the TurboFieldfare engine):
+ *  [LH] "Gemma 4 26B : Comment faire tourner un LLM en 2 Go de RAM",
+ *       section 04 "Implementation technique", parts "Le pipeline de
+ *       traitement" and "Concurrence pour masquer la latence".
+ *  [DS] daily.steinslab.io TurboFieldfare article, sections "L'atout cache
+ *       des modeles MoE" and "Trois optimisations cles" (items 1 and 3).
+ *  [RM] "TurboFieldfare execute Mac Gemma 4 26B dans 2 Go, mais la vitesse du
+ *       SSD devient le compromis", sections "Mac Gemma 4 26B tient en
+ *       memoire ..." and "L'affirmation des 2 Go ...".
+ *  [DT] "Een model met 26 miljard parameters uitvoeren in twee gigabyte
+ *       geheugen op een gewone Mac", section "Wat is de belangrijkste
+ *       architectuurtruuc".
+ *
+ * Conventions for every entry point:
+ *  - Every call returns an int status (MOE_OK or a negative MOE_ERR_*);
+ *    moe_last_error() returns a message for the calling thread's last error.
+ *  - Pointers marked "device" are CUDA device pointers on the current device;
+ *    "host" pointers are ordinary or pinned host memory as stated.
+ *  - The caller owns all buffers and streams.  The library allocates only in
+ *    moe_ctx_create (workspace, events, mapped host buffers) and frees them in
+ *    moe_ctx_destroy; no entry point allocates on the hot path.
+ *  - Calls are asynchronous on the given stream, except where a host wait is
+ *    stated.  One context serves one stream order at a time: calls on the
+ *    same context must not overlap on the GPU (they share its workspace).
+ *  - Every device pointer must be 16-byte aligned; sizes must satisfy the
+ *    limits of moe_ctx_create.  A violation returns an error and launches
+ *    nothing.
+ *  - fp16 values travel as their IEEE binary16 bit patterns (moe_half).
+ */
+#ifndef MOEQ4_H
+#define MOEQ4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_half;                 /* IEEE binary16 bits */
+typedef struct CUstream_st *moe_stream_t;  /* same handle as cudaStream_t */
+
+enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,      /* null pointer, bad count, bad flag */
+    MOE_ERR_ALIGNMENT = -2,        /* a pointer is not 16-byte aligned */
+    MOE_ERR_UNSUPPORTED_SHAPE = -3,/* sizes outside the supported limits */
+    MOE_ERR_CUDA = -4,             /* a CUDA runtime call failed */
+    MOE_ERR_TIMEOUT = -5,          /* a bounded device wait gave up */
+    MOE_ERR_CACHE_STATE = -6       /* LFU table invalid or fill failed */
+};
+
+enum { MOE_GELU_TANH = 0, MOE_GELU_ERF = 1 };
+
+/* Limits checked by every entry point. */
+enum {
+    MOE_MAX_TOPK = 8,
+    MOE_MAX_EXPERTS = 256,
+    MOE_MAX_SLOTS = 32,
+    MOE_GROUP = 64
+};
+
+/* Layer shape and switches.  hidden, inter and inter_shared are multiples of
+ * 64 (one quantisation group); top_k <= 8; n_experts <= 256;
+ * top_k < n_slots <= 32. */
+typedef struct {
+    int32_t hidden;        /* H  (2816 for the Gemma-like layer) */
+    int32_t n_experts;     /* E  routed experts (128) */
+    int32_t top_k;         /* k  experts per token (8) [DS], [LH] */
+    int32_t inter;         /* I  routed-expert intermediate (704) */
+    int32_t inter_shared;  /* Is shared-expert intermediate (2112) */
+    int32_t n_slots;       /* S  LFU slots per layer (16) [DS], [RM] */
+    int32_t renorm;        /* 1: routing weights renormalised over top-k */
+    int32_t gelu;          /* MOE_GELU_TANH or MOE_GELU_ERF */
+    double rms_eps;        /* RMSNorm epsilon (1e-6) */
+} MoeConfig;
+
+typedef struct moe_ctx moe_ctx;
+
+/* Creates a context for cfg on the current CUDA device, sized for up to
+ * max_tokens tokens per call.  Allocates its workspace, a mapped pinned host
+ * buffer for the streaming miss list, events and a device status word.
+ * Returns MOE_ERR_UNSUPPORTED_SHAPE when cfg breaks the limits above. */
+int moe_ctx_create(const MoeConfig *cfg, int max_tokens, moe_ctx **out);
+
+/* Synchronises the device and frees everything moe_ctx_create allocated.
+ * A null ctx is accepted. */
+int moe_ctx_destroy(moe_ctx *ctx);
+
+/* Message for the calling thread's most recent error ("" if none). */
+const char *moe_last_error(void);
+
+/* ------------------------------------------------------------ formats --
+ * Expert blob (one contiguous, 16-byte aligned buffer per expert; a blob is
+ * the unit of one cache fill):
+ *   [gate/up codes  u32 [2*inter][hidden/8]]  gate rows 0..inter-1,
+ *                                             up rows inter..2*inter-1
+ *   [gate/up scales fp16 [2*inter][hidden/64]]
+ *   [gate/up biases fp16 [2*inter][hidden/64]]
+ *   [down codes     u32 [hidden][inter/8]]
+ *   [down scales    fp16 [hidden][inter/64]]
+ *   [down biases    fp16 [hidden][inter/64]]
+ * Weight (row r, column c) = scale[r][c/64] * code + bias[r][c/64] with
+ * code = (word[r][c/8] >> 4*(c%8)) & 15: "MLX affine" 4-bit weights
+ * ([RM] "L'affirmation des 2 Go ..."; [DS] "Trois optimisations cles" 1).
+ * Router: int8 W[n_experts][hidden] with one fp16 scale per expert row
+ * (8-bit router: [LH] pipeline step 1; [DS] item 1).
+ */
+
+/* Size in bytes of one expert blob with the given hidden/intermediate. */
+size_t moe_blob_bytes(int hidden, int inter);
+
+/* ---------------------------------------------------------- router ----
+ * [LH] pipeline step 1, [DS] "L'atout cache des modeles MoE": for each of T
+ * tokens, logit_e = scale_e * sum_c W[e][c] * x[c] (+ bias_e), with the dot
+ * product of int8 weights and fp16 activations formed exactly in integer
+ * arithmetic and the epilogue in fp64; top_k experts by descending logit,
+ * ties to the lower index; weights = softmax over all E logits, then
+ * renormalised over the top_k when cfg.renorm.
+ *   Wr        device int8 [E][H]
+ *   row_scale device fp16 [E]
+ *   bias      device fp32 [E] or NULL
+ *   x         device fp16 [T][H]
+ *   topk_idx  device int32 [T][k]   (descending logit order)
+ *   topk_w    device fp32  [T][k]
+ *   logits    device fp64  [T][E] or NULL
+ * T must be 1..max_tokens. */
+int moe_router_topk(moe_ctx *ctx, const int8_t *Wr, const moe_half *row_scale,
+                    const float *bias, const moe_half *x, int T,
+                    int32_t *topk_idx, float *topk_w, double *logits,
+                    moe_stream_t stream);
+
+/* ----------------------------------------------------- expert FFN ----
+ * Grouped expert FFN over n_pairs (expert, token) pairs: for pair p,
+ *   g = Wg x, u = Wu x, h = GELU(g) * u, y[p] = Wd h,
+ * with x = row pairs[p].token of x, weights dequantised from the pair's
+ * blob, fp32 accumulation.  The GELU form is cfg.gelu.
+ *   pairs  device MoeFfnPair [n_pairs]; blob 16-byte aligned, inter equal
+ *          to cfg.inter or cfg.inter_shared, 0 <= token < T
+ *   x      device fp16 [T][H]
+ *   y      device fp32 [n_pairs][H]
+ * n_pairs must be 1..max_tokens*(top_k+1). */
+typedef struct {
+    const void *blob;   /* device expert blob */
+    int32_t inter;      /* its intermediate size */
+    int32_t token;      /* row of x */
+} MoeFfnPair;
+
+int moe_expert_ffn_q4(moe_ctx *ctx, const MoeFfnPair *pairs, int n_pairs,
+                      const moe_half *x, int T, float *y, moe_stream_t stream);
+
+/* --------------------------------------------------------- combine ----
+ * [LH] "Concurrence pour masquer la latence", [RM] "L'affirmation des 2 Go
+ * ...": the shared and routed outputs combine,
+ *   y_out[t] = y_shared[t] + sum_j topk_w[t][j] * y_routed[t][j]
+ * summed in j order in fp32.  When residual is not NULL,
+ *   residual[t][c] = fp16(float(residual[t][c]) + y_out[t][c]).
+ *   y_routed device fp32 [T][k][H]; y_shared device fp32 [T][H];
+ *   topk_w device fp32 [T][k]; y_out device fp32 [T][H];
+ *   residual device fp16 [T][H] or NULL. */
+int moe_combine(moe_ctx *ctx, const float *y_routed, const float *y_shared,
+                const float *topk_w, int T, float *y_out, moe_half *residual,
+                moe_stream_t stream);
+
+/* ------------------------------------------------------- LFU cache ----
+ * One layer's expert cache of n_slots slots ([DS] "Trois optimisations
+ * cles" item 3; [RM] "Mac Gemma 4 26B tient en memoire ..."), kept in device
+ * memory.  For each token in order:
+ *  (i)  its experts in ascending id order: a resident expert is a hit and its
+ *       count grows by one;
+ *  (ii) each missing expert in ascending id order takes the lowest empty
+ *       slot, else the slot not used by this token with the lowest count,
+ *       ties to the oldest insertion; it starts with count 1 and the next
+ *       insertion number.  A count does not survive eviction.
+ * Only the missing experts are fetched ([LH] pipeline step 3). */
+typedef struct {
+    int32_t expert[MOE_MAX_SLOTS];  /* resident expert, -1 when empty */
+    int64_t count[MOE_MAX_SLOTS];   /* uses since insertion */
+    int64_t seq[MOE_MAX_SLOTS];     /* insertion number */
+    int64_t counter;                /* last insertion number */
+    int64_t hits;                   /* running totals */
+    int64_t misses;
+    int32_t n_slots;
+    int32_t valid;                  /* 0 after a failed fill */
+} MoeLfuTable;
+
+/* Resets a device table to n_slots empty slots (top_k < n_slots <= 32). */
+int moe_lfu_init(moe_ctx *ctx, MoeLfuTable *table, int n_slots,
+                 moe_stream_t stream);
+
+/* Looks up T tokens' experts in order, updating the table.
+ *   table     device MoeLfuTable (valid)
+ *   topk_idx  device int32 [T][k]
+ *   slot_of   device int32 [T][k]: slot holding topk_idx[t][j] afterwards
+ *   miss_list device-visible int32 [T*k][2]: (expert, slot) per fill, in
+ *             fill order; may be mapped pinned host memory
+ *   n_miss    device-visible int32 [1]: number of fills, or -1 when the
+ *             table is invalid (nothing changed).
+ * When T > 1 a slot filled for token t may be evicted again by a later token
+ * of the same call; callers that fill after the call use T = 1. */
+int moe_cache_lookup_lfu(moe_ctx *ctx, MoeLfuTable *table,
+                         const int32_t *topk_idx, int T, int32_t *slot_of,
+                         int32_t *miss_list, int32_t *n_miss,
+                         moe_stream_t stream);
+
+/* -------------------------------------------------------- full layer ----
+ * One MoE layer for T tokens of one call ([LH] pipeline steps 1-4 and
+ * "Concurrence pour masquer la latence"; [RM] "L'affirmation des 2 Go ...";
+ * [DT] "Wat is de belangrijkste architectuurtruuc").
+ *
+ * Resident mode (layer->experts != NULL): router, grouped FFN of the shared
+ * and the routed experts, combine; all on `main`, no host wait.
+ *
+ * Streaming mode (layer->experts == NULL; host_store, slots, lfu set; T = 1):
+ * router and cache lookup on `main`, then the shared-expert FFN on `main`
+ * while the host waits for the miss list and issues one cudaMemcpyAsync per
+ * missing blob on `copy`; `main` waits for the copies, runs the routed FFN
+ * from the slots and combines.  The call returns after the copies are
+ * issued (one host wait per call).  If issuing a copy fails the table is
+ * marked invalid and MOE_ERR_CACHE_STATE is returned.
+ *
+ * flags & MOE_PRENORM: `x` is the fp16 residual stream h; the layer input is
+ * RMSNorm(h) (unit weight, eps = cfg.rms_eps, exact sum of squares, result
+ * rounded to fp16) and afterwards h <- fp16(h + y) in place.
+ */
+enum { MOE_PRENORM = 1 };
+
+typedef struct {
+    const int8_t *router_w;       /* device int8 [E][H] */
+    const moe_half *router_scale; /* device fp16 [E] */
+    const float *router_bias;     /* device fp32 [E] or NULL */
+    const void *shared_blob;      /* device blob (inter_shared) */
+    const void *experts;          /* resident: device [E] blobs, contiguous */
+    const void *host_store;       /* streaming: pinned host [E] blobs */
+    void *slots;                  /* streaming: device [n_slots] blobs */
+    MoeLfuTable *lfu;             /* streaming: device table */
+} MoeLayer;
+
+typedef struct {
+    float *y;              /* device fp32 [T][H]: MoE output, required */
+    int32_t *topk_idx;     /* device int32 [T][k] or NULL */
+    float *topk_w;         /* device fp32 [T][k] or NULL */
+    int32_t *slot_of;      /* device int32 [T][k] or NULL (streaming) */
+    moe_half *x_norm;      /* device fp16 [T][H] or NULL (MOE_PRENORM) */
+} MoeLayerOut;
+
+int moe_layer_decode(moe_ctx *ctx, const MoeLayer *layer, moe_half *x, int T,
+                     const MoeLayerOut *out, int flags, moe_stream_t main,
+                     moe_stream_t copy);
+
+/* ------------------------------------------------------------- stack ----
+ * Decodes T tokens one after another through n_layers resident layers
+ * (each token: for every layer, x = RMSNorm(h), y = MoE(x), h <- fp16(h+y)),
+ * the per-layer flow repeated over the layers and then per token ([RM]
+ * "L'affirmation des 2 Go ...").  The token loop runs as a captured CUDA
+ * graph replayed once per token; the first call for a given set of layers
+ * captures it.
+ *   layers  host array [n_layers] of resident MoeLayer
+ *   h       device fp16 [T][H], updated in place
+ *   y_last  device fp32 [T][H] or NULL: MoE output of the last layer */
+int moe_stack_decode(moe_ctx *ctx, const MoeLayer *layers, int n_layers,
+                     moe_half *h, int T, float *y_last, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOEQ4_H */

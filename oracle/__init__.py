@@ -68,6 +68,8 @@ def _load():
     lib.oracle_softmax.restype = None
     lib.oracle_topk_weights.argtypes = [P, P, i32, i32, P]
     lib.oracle_topk_weights.restype = None
+    lib.oracle_combine.argtypes = [P, P, P, i32, i32, P]
+    lib.oracle_combine.restype = None
     lib.oracle_moe_layer.argtypes = [i32, i32, i32, i32, i32, i32, i32,
                                      P, P, P, P, P, sz, P, P, P, P, P, P, P]
     lib.oracle_moe_layer.restype = None
@@ -168,6 +170,17 @@ def topk_weights(p, idx, renorm: int = 1):
     w = np.zeros(idx.size, np.float64)
     _load().oracle_topk_weights(_p(p), _p(idx), idx.size, int(renorm), _p(w))
     return w
+
+
+def combine(y_shared, y_routed, w):
+    """``oracle_combine``: y_shared [H], y_routed [k,H], w [k] -> y [H]."""
+    ys = _c(np.asarray(y_shared, np.float64), np.float64)
+    yr = _c(np.asarray(y_routed, np.float64), np.float64)
+    w = _c(np.asarray(w, np.float64), np.float64)
+    k, H = yr.shape
+    y = np.zeros(H, np.float64)
+    _load().oracle_combine(_p(ys), _p(yr), _p(w), k, H, _p(y))
+    return y
 
 
 def moe_layer(cfg, layer, x16):

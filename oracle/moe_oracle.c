@@ -255,6 +255,21 @@ void oracle_topk_weights(const double *p, const int32_t *idx, int k,
         w[j] = renorm ? p[idx[j]] / z : p[idx[j]];
 }
 
+/* ------------------------------------------------------------ combine */
+
+/* The shared and routed branch outputs combine with the routing weights:
+ *   y = y_shared + sum_j w_j y_routed[j]   (fp64). */
+void oracle_combine(const double *y_shared, const double *y_routed,
+                    const double *w, int k, int H, double *y)
+{
+    for (int c = 0; c < H; c++) {
+        double acc = y_shared[c];
+        for (int j = 0; j < k; j++)
+            acc += w[j] * y_routed[(size_t)j * (size_t)H + (size_t)c];
+        y[c] = acc;
+    }
+}
+
 /* ---------------------------------------------------------- MoE layer */
 
 /* One token through one MoE layer:
@@ -272,7 +287,6 @@ void oracle_moe_layer(int H, int E, int k, int I, int Is, int gelu, int renorm,
 {
     double *x = (double *)malloc(sizeof(double) * (size_t)H);
     double *p = (double *)malloc(sizeof(double) * (size_t)E);
-    double *ye = (double *)malloc(sizeof(double) * (size_t)H);
     for (int c = 0; c < H; c++)
         x[c] = oracle_half_to_double(x16[c]);
 
@@ -281,21 +295,21 @@ void oracle_moe_layer(int H, int E, int k, int I, int Is, int gelu, int renorm,
     oracle_softmax(logits, E, p);
     oracle_topk_weights(p, idx, k, renorm, w);
 
-    oracle_expert_ffn(shared_blob, H, Is, gelu, x, NULL, y);
-    if (y_shared)
-        memcpy(y_shared, y, sizeof(double) * (size_t)H);
-    for (int j = 0; j < k; j++) {
+    double *ys = (double *)malloc(sizeof(double) * (size_t)H);
+    double *yr = (double *)malloc(sizeof(double) * (size_t)H * (size_t)k);
+    oracle_expert_ffn(shared_blob, H, Is, gelu, x, NULL, ys);
+    for (int j = 0; j < k; j++)
         oracle_expert_ffn(expert_base + (size_t)idx[j] * blob_stride, H, I,
-                          gelu, x, NULL, ye);
-        if (y_routed)
-            memcpy(y_routed + (size_t)j * (size_t)H, ye,
-                   sizeof(double) * (size_t)H);
-        for (int c = 0; c < H; c++)
-            y[c] += w[j] * ye[c];
-    }
+                          gelu, x, NULL, yr + (size_t)j * (size_t)H);
+    oracle_combine(ys, yr, w, k, H, y);
+    if (y_shared)
+        memcpy(y_shared, ys, sizeof(double) * (size_t)H);
+    if (y_routed)
+        memcpy(y_routed, yr, sizeof(double) * (size_t)H * (size_t)k);
     free(x);
     free(p);
-    free(ye);
+    free(ys);
+    free(yr);
 }
 
 /* ------------------------------------------------------------- RMSNorm */

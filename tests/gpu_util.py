@@ -1,0 +1,53 @@
+"""Helpers shared by the GPU parity tests (no arithmetic of the method)."""
+import numpy as np
+import torch
+
+from bit_quantized_expert_int8_b200 import synth
+
+# Tolerance on fp32/fp64 layer outputs against the fp64 oracle.
+REL_L2 = 1e-3
+MAX_ABS = 2e-3
+
+
+def np_of(t):
+    if t is None:
+        return None
+    t = t.detach().cpu()
+    if t.dtype == torch.float16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def np_layer(d):
+    return {k: np_of(v) for k, v in d.items()}
+
+
+def to_dev(d, device="cuda"):
+    return {k: (None if v is None else v.to(device)) for k, v in d.items()}
+
+
+def assert_y_close(y_gpu, y_ref, what=""):
+    y_gpu = np.asarray(y_gpu, np.float64)
+    y_ref = np.asarray(y_ref, np.float64)
+    d = y_gpu - y_ref
+    rel = np.linalg.norm(d) / max(np.linalg.norm(y_ref), 1e-30)
+    mx = np.abs(d).max() if d.size else 0.0
+    assert rel <= REL_L2 and mx <= MAX_ABS, f"{what}: rel L2 {rel:.3e}, max abs {mx:.3e}"
+    return rel, mx
+
+
+def half_ulp_diff(a16, b16):
+    """Distance in fp16 units in the last place between two uint16 arrays."""
+    a = a16.astype(np.int32)
+    b = b16.astype(np.int32)
+    a = np.where(a & 0x8000, -(a & 0x7FFF), a)
+    b = np.where(b & 0x8000, -(b & 0x7FFF), b)
+    return np.abs(a - b)
+
+
+def make_layer(cfg, seed, layer=0, device="cuda", bias_std=None):
+    """Generate on the CPU for small shapes, on the GPU for large ones; the
+    oracle always receives a CPU copy of the very same bytes."""
+    gen_dev = "cpu" if cfg.H * cfg.I * cfg.E <= 2 ** 24 else device
+    d = synth.layer_weights(cfg, seed, layer, gen_dev, bias_std=bias_std)
+    return to_dev(d, device)

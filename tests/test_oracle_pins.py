@@ -229,6 +229,20 @@ def test_softmax_sums_to_one_and_matches_scipy():
     np.testing.assert_allclose(raw, sp_softmax(lg)[idx], rtol=1e-13)
 
 
+# -------------------------------------------------------------- combine ----
+
+def test_combine_special_cases():
+    rng = np.random.default_rng(8)
+    H, k = 96, 4
+    ys, yr = rng.standard_normal(H), rng.standard_normal((k, H))
+    np.testing.assert_array_equal(oracle.combine(ys, yr, np.zeros(k)), ys)
+    for j in range(k):
+        e = np.zeros(k); e[j] = 1.0
+        np.testing.assert_array_equal(oracle.combine(ys, yr, e), ys + yr[j])
+    w = rng.random(k)
+    np.testing.assert_allclose(oracle.combine(ys, yr, w), ys + w @ yr, rtol=1e-14, atol=1e-15)
+
+
 # ------------------------------------------------------------ MoE layer ----
 
 def _tiny_layer(cfg, seed=0, bias_std=None):
