@@ -46,6 +46,7 @@ static int fail(int code, const char* fmt, ...) {
     } while (0)
 
 static inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+static inline bool aligned4(const void* p) { return ((uintptr_t)p & 3u) == 0; }
 
 // ------------------------------------------------------------ context --
 struct StackKey {
@@ -248,9 +249,9 @@ extern "C" int moe_router_topk(moe_ctx* c, const int8_t* Wr, const moe_half* row
     if (!c || !Wr || !row_scale || !x || !topk_idx || !topk_w)
         return fail(MOE_ERR_INVALID_ARG, "moe_router_topk: NULL argument");
     if (T < 1 || T > c->maxT) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T=%d outside 1..%d", T, c->maxT);
-    if (!aligned16(Wr) || !aligned16(row_scale) || !aligned16(x) || !aligned16(topk_idx) ||
-        !aligned16(topk_w) || (bias && !aligned16(bias)) || (logits && !aligned16(logits)))
-        return fail(MOE_ERR_ALIGNMENT, "moe_router_topk: pointers must be 16-byte aligned");
+    if (!aligned16(Wr) || !aligned16(row_scale) || !aligned16(x) || !aligned4(topk_idx) ||
+        !aligned4(topk_w) || (bias && !aligned4(bias)) || (logits && !aligned16(logits)))
+        return fail(MOE_ERR_ALIGNMENT, "moe_router_topk: misaligned pointer");
     return launch_router(c, Wr, row_scale, bias, reinterpret_cast<const __half*>(x), T, topk_idx,
                          topk_w, logits, stream);
 }
@@ -274,9 +275,9 @@ extern "C" int moe_combine(moe_ctx* c, const float* y_routed, const float* y_sha
     if (!c || !y_routed || !y_shared || !topk_w || !y_out)
         return fail(MOE_ERR_INVALID_ARG, "moe_combine: NULL argument");
     if (T < 1 || T > 65535) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T=%d outside 1..65535", T);
-    if (!aligned16(y_routed) || !aligned16(y_shared) || !aligned16(topk_w) || !aligned16(y_out) ||
+    if (!aligned16(y_routed) || !aligned16(y_shared) || !aligned4(topk_w) || !aligned16(y_out) ||
         (residual && !aligned16(residual)))
-        return fail(MOE_ERR_ALIGNMENT, "moe_combine: pointers must be 16-byte aligned");
+        return fail(MOE_ERR_ALIGNMENT, "moe_combine: misaligned pointer");
     return launch_combine(c, y_routed, y_shared, topk_w, T, y_out,
                           reinterpret_cast<__half*>(residual), stream);
 }
@@ -297,8 +298,9 @@ extern "C" int moe_cache_lookup_lfu(moe_ctx* c, MoeLfuTable* table, const int32_
     if (!c || !table || !topk_idx || !slot_of || !miss_list || !n_miss)
         return fail(MOE_ERR_INVALID_ARG, "moe_cache_lookup_lfu: NULL argument");
     if (T < 1 || T > 65535) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T=%d outside 1..65535", T);
-    if (!aligned16(table) || !aligned16(topk_idx) || !aligned16(slot_of) || !aligned16(miss_list))
-        return fail(MOE_ERR_ALIGNMENT, "moe_cache_lookup_lfu: pointers must be 16-byte aligned");
+    if (!aligned16(table) || !aligned4(topk_idx) || !aligned4(slot_of) || !aligned4(miss_list) ||
+        !aligned4(n_miss))
+        return fail(MOE_ERR_ALIGNMENT, "moe_cache_lookup_lfu: misaligned pointer");
     k_lfu_lookup<<<1, 32, 0, stream>>>(table, topk_idx, T, c->cfg.top_k, slot_of, miss_list, n_miss);
     CKL();
     return MOE_OK;
@@ -395,8 +397,8 @@ extern "C" int moe_layer_decode(moe_ctx* c, const MoeLayer* L, moe_half* x, int 
     const void* ptrs[] = {L->router_w, L->router_scale, L->shared_blob, x, o->y};
     for (const void* p : ptrs)
         if (!aligned16(p)) return fail(MOE_ERR_ALIGNMENT, "moe_layer_decode: pointers must be 16-byte aligned");
-    if ((L->router_bias && !aligned16(L->router_bias)) || (o->topk_idx && !aligned16(o->topk_idx)) ||
-        (o->topk_w && !aligned16(o->topk_w)) || (o->slot_of && !aligned16(o->slot_of)) ||
+    if ((L->router_bias && !aligned4(L->router_bias)) || (o->topk_idx && !aligned4(o->topk_idx)) ||
+        (o->topk_w && !aligned4(o->topk_w)) || (o->slot_of && !aligned4(o->slot_of)) ||
         (o->x_norm && !aligned16(o->x_norm)))
         return fail(MOE_ERR_ALIGNMENT, "moe_layer_decode: pointers must be 16-byte aligned");
     if (L->experts) {
@@ -427,7 +429,7 @@ extern "C" int moe_stack_decode(moe_ctx* c, const MoeLayer* layers, int n_layers
         if (!L.router_w || !L.router_scale || !L.shared_blob || !L.experts)
             return fail(MOE_ERR_INVALID_ARG, "layer %d is not a resident layer", l);
         if (!aligned16(L.router_w) || !aligned16(L.router_scale) || !aligned16(L.shared_blob) ||
-            !aligned16(L.experts) || (L.router_bias && !aligned16(L.router_bias)))
+            !aligned16(L.experts) || (L.router_bias && !aligned4(L.router_bias)))
             return fail(MOE_ERR_ALIGNMENT, "layer %d: pointers must be 16-byte aligned", l);
     }
     const int H = c->cfg.hidden;

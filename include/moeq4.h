@@ -31,7 +31,9 @@
  *  - Calls are asynchronous on the given stream, except where a host wait is
  *    stated.  One context serves one stream order at a time: calls on the
  *    same context must not overlap on the GPU (they share its workspace).
- *  - Every device pointer must be 16-byte aligned; sizes must satisfy the
+ *  - Weight, blob, activation and output-row pointers must be 16-byte
+ *    aligned; int32/fp32 index and weight arrays (topk_idx, topk_w, slot_of,
+ *    miss_list, n_miss, router bias) need 4 bytes.  Sizes must satisfy the
  *    limits of moe_ctx_create.  A violation returns an error and launches
  *    nothing.
  *  - fp16 values travel as their IEEE binary16 bit patterns (moe_half).
@@ -52,7 +54,7 @@ typedef struct CUstream_st *moe_stream_t;  /* same handle as cudaStream_t */
 enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = -1,      /* null pointer, bad count, bad flag */
-    MOE_ERR_ALIGNMENT = -2,        /* a pointer is not 16-byte aligned */
+    MOE_ERR_ALIGNMENT = -2,        /* a pointer is misaligned */
     MOE_ERR_UNSUPPORTED_SHAPE = -3,/* sizes outside the supported limits */
     MOE_ERR_CUDA = -4,             /* a CUDA runtime call failed */
     MOE_ERR_TIMEOUT = -5,          /* a bounded device wait gave up */
