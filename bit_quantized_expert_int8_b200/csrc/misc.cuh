@@ -161,6 +161,10 @@ __global__ void k_copy_half_row(const __half* __restrict__ src, __half* __restri
     for (int c = threadIdx.x; c < H; c += blockDim.x) d[c] = s[c];
 }
 
+__global__ void k_copy_rows(const __half* __restrict__ src, __half* __restrict__ dst, int n) {
+    for (int c = threadIdx.x; c < n; c += blockDim.x) dst[c] = src[c];
+}
+
 __global__ void k_store_token(const __half* __restrict__ h_cur, const float* __restrict__ y,
                               __half* __restrict__ h_all, float* __restrict__ y_all,
                               int* __restrict__ cursor, int H) {

@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "ffn_simple.cuh"
+#include "layer_fused.cuh"
 #include "misc.cuh"
 #include "router.cuh"
 
@@ -87,6 +88,19 @@ struct moe_ctx {
     // host-side fault injection (tests): fail the Nth blob copy before issue
     long fail_copy_at = -1;
     long copies_seen = 0;
+    // fused single-token layer kernel
+    FusedSync* fsync = nullptr;        // [4 modes][2 parities]
+    int* status = nullptr;             // device status word (bounded waits)
+    __half* h_alt = nullptr;           // ping-pong residual buffer
+    int fparity[4] = {0, 0, 0, 0};
+    int n_sms = 0;
+    bool fused_ok = false;
+    uint32_t* dlimb = nullptr;         // packed intermediate of the fused kernel
+    int f_stages = 0, f_stage_bytes = 0;
+    unsigned long long* trace = nullptr;   // [n_sms * 16] phase stamps
+    bool tracing = false;
+    size_t f_smem = 0;
+    void (*f_kernel)(const FusedArgs) = nullptr;
 };
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -132,6 +146,41 @@ extern "C" int moe_ctx_destroy(moe_ctx* c) {
     return MOE_OK;
 }
 
+// Chooses the fused kernel variant and its shared-memory ring for cfg.
+static cudaError_t setup_fused(moe_ctx* c) {
+    const MoeConfig& g = c->cfg;
+    int dev = c->device, optin = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&c->n_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    const int nch = g.hidden / 32;
+    const int maxc = (nch + 31) / 32;
+    const int NC = (g.top_k * g.inter + g.inter_shared) / 32;
+    const int maxd = (NC + 255) / 256;
+    size_t stage = (size_t)18 * g.hidden;                          // gate/up item
+    const size_t down = (size_t)9 * ((size_t)g.top_k * g.inter + g.inter_shared) / 2;
+    if (down > stage) stage = down;
+    stage = (stage + 127) / 128 * 128;
+    int ns = 0;
+    for (int n = kFusedMaxStages; n >= 2 && ns == 0; n--)
+        if ((size_t)n * stage + fused_fixed_smem(g.hidden, n) <= (size_t)optin) ns = n;
+    c->fused_ok = g.hidden <= 4096 && maxc >= 1 && maxc <= 4 && maxd >= 1 && maxd <= 2 &&
+                  ns >= 2 && stage < (1u << 20) && c->n_sms > 0;
+    if (!c->fused_ok) return cudaSuccess;
+    typedef void (*KFn)(const FusedArgs);
+    static const KFn table[4][2] = {
+        {k_moe_layer_fused<1, 1>, k_moe_layer_fused<1, 2>},
+        {k_moe_layer_fused<2, 1>, k_moe_layer_fused<2, 2>},
+        {k_moe_layer_fused<3, 1>, k_moe_layer_fused<3, 2>},
+        {k_moe_layer_fused<4, 1>, k_moe_layer_fused<4, 2>}};
+    c->f_kernel = table[maxc - 1][maxd - 1];
+    c->f_stages = ns;
+    c->f_stage_bytes = (int)stage;
+    c->f_smem = (size_t)ns * stage + fused_fixed_smem(g.hidden, ns);
+    return cudaFuncSetAttribute(c->f_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)c->f_smem);
+}
+
 extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** out) {
     if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
     *out = nullptr;
@@ -159,6 +208,13 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     size_t o_cur = take(sizeof(int));
     size_t o_hcur = take(H * sizeof(__half));
     size_t o_ycur = take(H * sizeof(float));
+    size_t o_fsync = take(8 * sizeof(FusedSync));
+    size_t o_status = take(sizeof(int));
+    size_t o_halt = take(H * sizeof(__half));
+    size_t o_dlimb = take((k * (size_t)cfg->inter + cfg->inter_shared) / 32 * kDLimbWords * 4);
+    int n_sms_dev = 0;
+    cudaDeviceGetAttribute(&n_sms_dev, cudaDevAttrMultiProcessorCount, c->device);
+    size_t o_trace = take((size_t)(n_sms_dev > 0 ? n_sms_dev : 1) * kTraceWords * sizeof(unsigned long long));
     int rc = MOE_OK;
     cudaError_t e = cudaMalloc(&c->ws, off);
     if (e == cudaSuccess) e = cudaMemset(c->ws, 0, off);
@@ -175,6 +231,11 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
         c->cursor = (int*)(c->ws + o_cur);
         c->h_cur = (__half*)(c->ws + o_hcur);
         c->y_cur = (float*)(c->ws + o_ycur);
+        c->fsync = (FusedSync*)(c->ws + o_fsync);
+        c->status = (int*)(c->ws + o_status);
+        c->h_alt = (__half*)(c->ws + o_halt);
+        c->dlimb = (uint32_t*)(c->ws + o_dlimb);
+        c->trace = (unsigned long long*)(c->ws + o_trace);
         size_t nm = T * k * 2 + 4;
         e = cudaHostAlloc((void**)&c->miss_host, nm * sizeof(int32_t), cudaHostAllocMapped);
     }
@@ -195,6 +256,7 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_ffn_down_simple, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)(c->maxI * sizeof(float)));
+    if (e == cudaSuccess) e = setup_fused(c);
     if (e != cudaSuccess) {
         rc = fail(MOE_ERR_CUDA, "moe_ctx_create: %s", cudaGetErrorString(e));
         moe_ctx_destroy(c);
@@ -239,6 +301,62 @@ static int launch_combine(moe_ctx* c, const float* y_routed, const float* y_shar
     k_combine<<<grid, 256, 0, s>>>(y_routed, (size_t)g.top_k * g.hidden, y_shared, g.hidden, w,
                                    g.top_k, g.hidden, y, residual);
     CKL();
+    return MOE_OK;
+}
+
+// One token through one layer with the fused kernel.  `mode` selects the
+// work classes of this launch (kModeFull for a resident layer; streaming
+// splits it into router / shared / routed+down launches).  Routed blobs are
+// experts + sel[j] * stride with sel = the routing indices, or the cache
+// slots when `sel_slots` is given.
+static int launch_fused(moe_ctx* c, const MoeLayer* L, const __half* x_in, __half* h_out,
+                        __half* x_norm_out, float* y, int32_t* idx_out, float* w_out,
+                        int prenorm, cudaStream_t s, int mode = kModeFull,
+                        const void* experts = nullptr, const int32_t* sel_slots = nullptr) {
+    const MoeConfig& g = c->cfg;
+    const int mi = mode == kModeFull ? 0 : mode == kModeRouter ? 1 : mode == kModeShared ? 2 : 3;
+    FusedArgs a{};
+    a.Wr = L->router_w;
+    a.rscale = reinterpret_cast<const __half*>(L->router_scale);
+    a.rbias = L->router_bias;
+    a.shared = static_cast<const uint8_t*>(L->shared_blob);
+    a.experts = static_cast<const uint8_t*>(experts ? experts : L->experts);
+    a.stride = BlobLayout(g.hidden, g.inter).bytes;
+    a.sel_src = sel_slots ? sel_slots : c->idx;
+    a.x_in = x_in;
+    a.h_out = h_out;
+    a.x_norm_out = x_norm_out;
+    a.y = y;
+    a.idx_ws = c->idx;
+    a.w_ws = c->w;
+    a.idx_out = idx_out;
+    a.w_out = w_out;
+    a.logits = c->logits;
+    a.dlimb = c->dlimb;
+    a.sync = c->fsync + 2 * mi + c->fparity[mi];
+    c->fparity[mi] ^= 1;
+    a.status = c->status;
+    a.trace = c->tracing ? c->trace : nullptr;
+    a.eps = g.rms_eps;
+    a.H = g.hidden; a.E = g.n_experts; a.k = g.top_k; a.I = g.inter; a.Is = g.inter_shared;
+    a.gelu = g.gelu; a.renorm = g.renorm; a.prenorm = prenorm;
+    a.n_stages = c->f_stages; a.stage_bytes = c->f_stage_bytes;
+    a.NR = (mode & kModeRouter) ? (g.n_experts + kRouterRows - 1) / kRouterRows : 0;
+    a.NSG = (mode & kModeShared) ? g.inter_shared / kGuRows : 0;
+    a.NRG = (mode & kModeRouted) ? g.top_k * (g.inter / kGuRows) : 0;
+    a.ND = (mode & kModeDown) ? g.hidden / 8 : 0;
+    a.NTOT = a.NR + a.NSG + a.NRG + a.ND;
+    cudaLaunchConfig_t lc{};
+    lc.gridDim = dim3(c->n_sms);
+    lc.blockDim = dim3(kFusedThreads);
+    lc.dynamicSmemBytes = c->f_smem;
+    lc.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    CK(cudaLaunchKernelEx(&lc, c->f_kernel, a));
     return MOE_OK;
 }
 
@@ -311,6 +429,17 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
                           int flags, cudaStream_t s) {
     const MoeConfig& g = c->cfg;
     const int k = g.top_k, H = g.hidden;
+    if (T == 1 && c->fused_ok) {
+        const bool pre = (flags & MOE_PRENORM) != 0;
+        TRY(launch_fused(c, L, x, pre ? c->h_alt : nullptr,
+                         reinterpret_cast<__half*>(o->x_norm), o->y, o->topk_idx, o->topk_w,
+                         pre ? 1 : 0, s));
+        if (pre) {
+            k_copy_rows<<<1, 256, 0, s>>>(c->h_alt, x, H);
+            CKL();
+        }
+        return MOE_OK;
+    }
     const __half* xin = x;
     __half* xn = o->x_norm ? reinterpret_cast<__half*>(o->x_norm) : c->x_norm;
     if (flags & MOE_PRENORM) {
@@ -333,8 +462,61 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
     return MOE_OK;
 }
 
+// Issues one cudaMemcpyAsync per missing blob on the copy stream (after the
+// host has waited for the miss list); marks the table invalid on failure.
+static int issue_fills(moe_ctx* c, const MoeLayer* L, cudaStream_t s, cudaStream_t cs) {
+    const size_t stride = BlobLayout(c->cfg.hidden, c->cfg.inter).bytes;
+    CK(cudaEventSynchronize(c->ev_lookup));
+    const int nm = *(volatile int32_t*)c->n_miss_host;
+    if (nm < 0) return fail(MOE_ERR_CACHE_STATE, "LFU table is invalid (an earlier fill failed)");
+    const uint8_t* store = static_cast<const uint8_t*>(L->host_store);
+    uint8_t* slots = static_cast<uint8_t*>(L->slots);
+    for (int i = 0; i < nm; i++) {
+        const int e = c->miss_host[2 * i], slot = c->miss_host[2 * i + 1];
+        cudaError_t err = cudaSuccess;
+        if (c->fail_copy_at >= 0 && c->copies_seen == c->fail_copy_at) err = cudaErrorInvalidValue;
+        c->copies_seen++;
+        if (err == cudaSuccess)
+            err = cudaMemcpyAsync(slots + (size_t)slot * stride, store + (size_t)e * stride, stride,
+                                  cudaMemcpyHostToDevice, cs);
+        if (err != cudaSuccess) {
+            k_lfu_invalidate<<<1, 1, 0, s>>>(L->lfu);
+            return fail(MOE_ERR_CACHE_STATE, "fill of expert %d into slot %d failed: %s; table "
+                        "marked invalid", e, slot, cudaGetErrorString(err));
+        }
+    }
+    CK(cudaEventRecord(c->ev_copy, cs));
+    CK(cudaStreamWaitEvent(s, c->ev_copy, 0));
+    return MOE_OK;
+}
+
+// Streaming layer with the fused kernel: router launch, cache lookup, shared
+// branch launch overlapping the fills, then routed + down launch reading the
+// slots.  Same arithmetic as the resident fused launch, so identical output.
+static int layer_streaming_fused(moe_ctx* c, const MoeLayer* L, __half* x, const MoeLayerOut* o,
+                                 int flags, cudaStream_t s, cudaStream_t cs) {
+    const MoeConfig& g = c->cfg;
+    const int pre = (flags & MOE_PRENORM) ? 1 : 0;
+    int32_t* slot_of = o->slot_of ? o->slot_of : c->slot_of;
+    TRY(launch_fused(c, L, x, nullptr, reinterpret_cast<__half*>(o->x_norm), nullptr, o->topk_idx,
+                     o->topk_w, pre, s, kModeRouter));
+    k_lfu_lookup<<<1, 32, 0, s>>>(L->lfu, c->idx, 1, g.top_k, slot_of, c->miss_dev, c->n_miss_dev);
+    CKL();
+    CK(cudaEventRecord(c->ev_lookup, s));
+    TRY(launch_fused(c, L, x, nullptr, nullptr, nullptr, nullptr, nullptr, pre, s, kModeShared));
+    TRY(issue_fills(c, L, s, cs));
+    TRY(launch_fused(c, L, x, pre ? c->h_alt : nullptr, nullptr, o->y, nullptr, nullptr, pre, s,
+                     kModeRouted | kModeDown, L->slots, slot_of));
+    if (pre) {
+        k_copy_rows<<<1, 256, 0, s>>>(c->h_alt, x, g.hidden);
+        CKL();
+    }
+    return MOE_OK;
+}
+
 static int layer_streaming(moe_ctx* c, const MoeLayer* L, __half* x, const MoeLayerOut* o,
                            int flags, cudaStream_t s, cudaStream_t cs) {
+    if (c->fused_ok) return layer_streaming_fused(c, L, x, o, flags, s, cs);
     const MoeConfig& g = c->cfg;
     const int k = g.top_k, H = g.hidden, T = 1;
     const __half* xin = x;
@@ -358,27 +540,7 @@ static int layer_streaming(moe_ctx* c, const MoeLayer* L, __half* x, const MoeLa
     CKL();
     // shared branch computes while the misses are fetched
     TRY(launch_ffn(c, c->pairs, T, xin, T, c->h_ws, c->y_pairs, s));
-    CK(cudaEventSynchronize(c->ev_lookup));
-    const int nm = *(volatile int32_t*)c->n_miss_host;
-    if (nm < 0) return fail(MOE_ERR_CACHE_STATE, "LFU table is invalid (an earlier fill failed)");
-    const uint8_t* store = static_cast<const uint8_t*>(L->host_store);
-    uint8_t* slots = static_cast<uint8_t*>(L->slots);
-    for (int i = 0; i < nm; i++) {
-        const int e = c->miss_host[2 * i], slot = c->miss_host[2 * i + 1];
-        cudaError_t err = cudaSuccess;
-        if (c->fail_copy_at >= 0 && c->copies_seen == c->fail_copy_at) err = cudaErrorInvalidValue;
-        c->copies_seen++;
-        if (err == cudaSuccess)
-            err = cudaMemcpyAsync(slots + (size_t)slot * stride, store + (size_t)e * stride, stride,
-                                  cudaMemcpyHostToDevice, cs);
-        if (err != cudaSuccess) {
-            k_lfu_invalidate<<<1, 1, 0, s>>>(L->lfu);
-            return fail(MOE_ERR_CACHE_STATE, "fill of expert %d into slot %d failed: %s; table "
-                        "marked invalid", e, slot, cudaGetErrorString(err));
-        }
-    }
-    CK(cudaEventRecord(c->ev_copy, cs));
-    CK(cudaStreamWaitEvent(s, c->ev_copy, 0));
+    TRY(issue_fills(c, L, s, cs));
     TRY(launch_ffn(c, c->pairs + T, T * k, xin, T, c->h_ws + (size_t)T * c->maxI,
                    c->y_pairs + (size_t)T * H, s));
     TRY(launch_combine(c, c->y_pairs + (size_t)T * H, c->y_pairs, w, T, o->y,
@@ -413,6 +575,37 @@ extern "C" int moe_layer_decode(moe_ctx* c, const MoeLayer* L, moe_half* x, int 
     return layer_streaming(c, L, reinterpret_cast<__half*>(x), o, flags, main, copy);
 }
 
+extern "C" int moe_ctx_check(moe_ctx* c, moe_stream_t stream) {
+    if (!c) return fail(MOE_ERR_INVALID_ARG, "moe_ctx_check: NULL context");
+    CK(cudaStreamSynchronize(stream));
+    int st = 0;
+    CK(cudaMemcpy(&st, c->status, sizeof(int), cudaMemcpyDeviceToHost));
+    if (st == 0) return MOE_OK;
+    // a bounded wait gave up: clear the status and the launch counters so the
+    // context can be used again
+    CK(cudaMemset(c->status, 0, sizeof(int)));
+    CK(cudaMemset(c->fsync, 0, 8 * sizeof(FusedSync)));
+    for (int m = 0; m < 4; m++) c->fparity[m] = 0;
+    return fail(st, "a bounded device wait gave up (status %d); counters reset", st);
+}
+
+extern "C" int moe_ctx_trace(moe_ctx* c, int enable, unsigned long long* host_out,
+                             int max_words) {
+    if (!c) return fail(MOE_ERR_INVALID_ARG, "moe_ctx_trace: NULL context");
+    const int words = c->n_sms * kTraceWords;
+    int n = 0;
+    if (host_out) {
+        CK(cudaDeviceSynchronize());
+        n = max_words < words ? max_words : words;
+        if (n > 0) CK(cudaMemcpy(host_out, c->trace, (size_t)n * 8, cudaMemcpyDeviceToHost));
+    }
+    if (enable >= 0) {
+        if (enable && !c->tracing) CK(cudaMemset(c->trace, 0, (size_t)words * 8));
+        c->tracing = enable != 0;
+    }
+    return n;
+}
+
 static bool same_key(const StackKey& k, const MoeLayer* layers, int n, moe_half* h, float* y) {
     if ((int)k.layers.size() != n || k.h != h || k.y_last != y) return false;
     return memcmp(k.layers.data(), layers, sizeof(MoeLayer) * n) == 0;
@@ -441,10 +634,18 @@ extern "C" int moe_stack_decode(moe_ctx* c, const MoeLayer* layers, int n_layers
         k_copy_half_row<<<1, 256, 0, cs>>>(reinterpret_cast<__half*>(h), c->h_cur, c->cursor, H, 1);
         MoeLayerOut o{};
         o.y = c->y_cur;
-        for (int l = 0; l < n_layers && rc == MOE_OK; l++)
-            rc = layer_resident(c, &layers[l], c->h_cur, 1, &o, MOE_PRENORM, cs);
+        __half* cur = c->h_cur;
+        for (int l = 0; l < n_layers && rc == MOE_OK; l++) {
+            if (c->fused_ok) {
+                __half* nxt = cur == c->h_cur ? c->h_alt : c->h_cur;
+                rc = launch_fused(c, &layers[l], cur, nxt, nullptr, c->y_cur, nullptr, nullptr, 1, cs);
+                cur = nxt;
+            } else {
+                rc = layer_resident(c, &layers[l], c->h_cur, 1, &o, MOE_PRENORM, cs);
+            }
+        }
         if (rc == MOE_OK)
-            k_store_token<<<1, 256, 0, cs>>>(c->h_cur, c->y_cur, reinterpret_cast<__half*>(h), y_last,
+            k_store_token<<<1, 256, 0, cs>>>(cur, c->y_cur, reinterpret_cast<__half*>(h), y_last,
                                              c->cursor, H);
         cudaGraph_t graph = nullptr;
         cudaError_t e = cudaStreamEndCapture(cs, &graph);

@@ -27,7 +27,8 @@ MOE_ERR_CACHE_STATE = -6
 MOE_PRENORM = 1
 MOE_MAX_SLOTS = 32
 
-EXPORTS = ("moe_ctx_create", "moe_ctx_destroy", "moe_last_error", "moe_blob_bytes",
+EXPORTS = ("moe_ctx_create", "moe_ctx_destroy", "moe_ctx_check", "moe_ctx_trace",
+           "moe_last_error", "moe_blob_bytes",
            "moe_router_topk", "moe_expert_ffn_q4", "moe_combine", "moe_lfu_init",
            "moe_cache_lookup_lfu", "moe_layer_decode", "moe_stack_decode")
 
@@ -67,6 +68,7 @@ class CMoeLfuTable(ctypes.Structure):
 
 LFU_TABLE_BYTES = ctypes.sizeof(CMoeLfuTable)
 PAIR_BYTES = 16   # MoeFfnPair: blob pointer, int32 inter, int32 token
+TRACE_WORDS = 160  # per CTA trace record of the fused layer kernel
 
 _lib = None
 
@@ -84,6 +86,8 @@ def load() -> ctypes.CDLL:
     sig = {
         "moe_ctx_create": ([ctypes.POINTER(CMoeConfig), i32, ctypes.POINTER(P)], i32),
         "moe_ctx_destroy": ([P], i32),
+        "moe_ctx_check": ([P, P], i32),
+        "moe_ctx_trace": ([P, i32, P, i32], i32),
         "moe_last_error": ([], ctypes.c_char_p),
         "moe_blob_bytes": ([i32, i32], ctypes.c_size_t),
         "moe_router_topk": ([P, P, P, P, P, i32, P, P, P, P], i32),
@@ -155,6 +159,26 @@ class Context:
             self.close()
         except Exception:
             pass
+
+
+def moe_ctx_check(ctx, stream=None):
+    """Synchronise and raise MoeError(MOE_ERR_TIMEOUT) if a bounded device
+    wait of this context gave up since the last check."""
+    _check(load().moe_ctx_check(ctx.handle, _stream(stream)))
+
+
+def moe_ctx_trace(ctx, enable=-1, read=False):
+    """Switch phase tracing of the fused layer kernel (1 on, 0 off, -1 keep);
+    with read=True return the last launch's records as an int64 array
+    [n_ctas, 16] (see moeq4.h)."""
+    import numpy as np
+    n = 1024 * TRACE_WORDS
+    buf = np.zeros(n, dtype=np.uint64) if read else None
+    rc = load().moe_ctx_trace(ctx.handle, int(enable),
+                              buf.ctypes.data if read else None, n if read else 0)
+    if rc < 0:
+        _check(rc)
+    return buf[:rc].reshape(-1, TRACE_WORDS) if read else None
 
 
 def moe_router_topk(ctx, Wr, row_scale, bias, x, T, topk_idx, topk_w, logits=None, stream=None):

@@ -98,6 +98,24 @@ int moe_ctx_create(const MoeConfig *cfg, int max_tokens, moe_ctx **out);
  * A null ctx is accepted. */
 int moe_ctx_destroy(moe_ctx *ctx);
 
+/* Synchronises `stream` and reports whether any kernel of this context gave
+ * up a bounded device wait since the last check (MOE_ERR_TIMEOUT, with the
+ * context's counters reset so that it can be used again) or MOE_OK. */
+int moe_ctx_check(moe_ctx *ctx, moe_stream_t stream);
+
+/* Tracing of the single-token layer kernel.  enable = 1 makes later launches
+ * record, per CTA, 160 words: globaltimer stamps (ns) of kernel entry, end of
+ * the input prologue, first item, routing known, down phase ready, consumer
+ * end, producer end, top-k published; word 8 counts router / shared /
+ * routed / down items in 16-bit fields; word 9 is the SM id; words 10-18
+ * router item done, top-k start and steps, prologue steps; words 32.. hold,
+ * for the CTA's first 42 items, three stamps each (copies issued, data
+ * ready, item done): time in the low 56 bits, item type + 1 in bits 56-59.  enable = 0
+ * stops recording, -1 leaves it as is.  When host_out is not NULL the device
+ * is synchronised and up to max_words words of the last recorded launch are
+ * copied; returns the number of words copied (>= 0) or an error. */
+int moe_ctx_trace(moe_ctx *ctx, int enable, unsigned long long *host_out, int max_words);
+
 /* Message for the calling thread's most recent error ("" if none). */
 const char *moe_last_error(void);
 

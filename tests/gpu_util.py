@@ -45,6 +45,16 @@ def half_ulp_diff(a16, b16):
     return np.abs(a - b)
 
 
+def assert_half_close(h_gpu16, h_ref16, what=""):
+    """fp16 residual check: |gpu - ref| <= 1 ulp of ref + the y tolerance
+    (h + y can cancel, where ulps of a tiny result say nothing)."""
+    g = np.asarray(h_gpu16).view(np.float16).astype(np.float64)
+    r = np.asarray(h_ref16).view(np.float16).astype(np.float64)
+    ulp = np.spacing(np.abs(r).astype(np.float16)).astype(np.float64)
+    bad = np.abs(g - r) > ulp + MAX_ABS
+    assert not bad.any(), f"{what}: {bad.sum()} residual entries off, worst {np.abs(g - r).max():.3e}"
+
+
 def make_layer(cfg, seed, layer=0, device="cuda", bias_std=None):
     """Generate on the CPU for small shapes, on the GPU for large ones; the
     oracle always receives a CPU copy of the very same bytes."""

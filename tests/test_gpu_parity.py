@@ -11,7 +11,7 @@ import torch
 import oracle
 from bit_quantized_expert_int8_b200 import build, moeq4, synth
 from bit_quantized_expert_int8_b200.config import LAYER, TINY, MoeConfig
-from gpu_util import (assert_y_close, half_ulp_diff, make_layer, np_layer, np_of)
+from gpu_util import (assert_half_close, assert_y_close, make_layer, np_layer, np_of)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -127,7 +127,7 @@ def test_combine_parity_and_residual():
                              w[t].cpu().double().numpy())
         assert_y_close(y[t].cpu().numpy(), ref)
         href = oracle.residual_add(h0[t], ref)
-        assert half_ulp_diff(np_of(h)[t], href).max() <= 1
+        assert_half_close(np_of(h)[t], href)
 
 
 # ------------------------------------------------------------------- LFU ----
@@ -227,7 +227,7 @@ def test_layer_prenorm_rmsnorm_exact_and_residual():
         assert idx[t].cpu().tolist() == ref["idx"].tolist()
         assert_y_close(y[t].cpu().numpy(), ref["y"])
         href = oracle.residual_add(h0[t], ref["y"])
-        assert half_ulp_diff(np_of(h)[t], href).max() <= 1
+        assert_half_close(np_of(h)[t], href)
 
 
 # ------------------------------------------------------------------- stack ----
