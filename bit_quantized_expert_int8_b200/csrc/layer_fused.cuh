@@ -309,21 +309,12 @@ __device__ __forceinline__ unsigned long long order_key(double d) {
     return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
 
-__device__ __forceinline__ void fused_topk_publish(const FusedArgs& a, unsigned long long epoch,
-                                                   int lane) {
+// Exact selection by rounds of three max-reductions over the 64-bit keys.
+__device__ __forceinline__ void topk_exact_rounds(const FusedArgs& a, const double* v,
+                                                  const unsigned long long* key, int lane,
+                                                  int& sel, double& sel_l, double& m) {
     constexpr int kPer = MOE_MAX_EXPERTS / 32;
-    double v[kPer];
-    unsigned long long key[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; i++) {
-        const int e = lane + 32 * i;
-        v[i] = e < a.E ? __ldcg(a.logits + e) : 0.0;
-        key[i] = e < a.E ? order_key(v[i]) : 0ull;      // 0 sorts below every logit
-    }
-    if (lane == 0) fused_trace(a, kTrTopkLoaded);
     unsigned taken = 0;
-    int sel = 0;
-    double sel_l = 0.0, m = 0.0;
     for (int j = 0; j < a.k; j++) {
         unsigned long long bk = 0;
         int bi = 0;
@@ -342,6 +333,78 @@ __device__ __forceinline__ void fused_topk_publish(const FusedArgs& a, unsigned 
         if (lane == wl) taken |= 1u << (wi >> 5);
         if (j == 0) m = wv;
         if (lane == j) { sel = (int)wi; sel_l = wv; }
+    }
+}
+
+// Top-k of logits[0..E), largest first, ties to the lower index, then the
+// softmax weights of the selected experts, published as the launch's tagged
+// routing record and to the caller's outputs.  Fast path: one max-reduction
+// per round on (24-bit order key << 8 | 255 - index); the 24-bit key is a
+// monotone function of the logit, so every expert whose key beats the k-th
+// pick's key is in the exact top-k and every expert below it is out; when no
+// other expert shares the k-th key the picked set is exact, and its order is
+// then settled by exact fp64 comparisons.  Otherwise the exact rounds run.
+__device__ __forceinline__ void fused_topk_publish(const FusedArgs& a, unsigned long long epoch,
+                                                   int lane) {
+    constexpr int kPer = MOE_MAX_EXPERTS / 32;
+    double v[kPer];
+    unsigned long long key[kPer];
+    unsigned pk[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; i++) {
+        const int e = lane + 32 * i;
+        v[i] = e < a.E ? __ldcg(a.logits + e) : 0.0;
+        key[i] = e < a.E ? order_key(v[i]) : 0ull;      // 0 sorts below every logit
+        pk[i] = e < a.E ? ((unsigned)(key[i] >> 40) << 8) | (unsigned)(255 - e) : 0u;
+    }
+    if (lane == 0) fused_trace(a, kTrTopkLoaded);
+    unsigned taken = 0, last = 0;
+    int sel = 0;
+    double sel_l = 0.0;
+    for (int j = 0; j < a.k; j++) {
+        unsigned best = 0;
+#pragma unroll
+        for (int i = 0; i < kPer; i++)
+            if (!((taken >> i) & 1u) && pk[i] > best) best = pk[i];
+        const unsigned w = __reduce_max_sync(0xffffffffu, best);
+        const unsigned wi = 255u - (w & 255u);
+        const int wl = (int)(wi & 31u);
+        double wv = 0.0;
+#pragma unroll
+        for (int i = 0; i < kPer; i++)
+            if ((unsigned)(lane + 32 * i) == wi) wv = v[i];
+        wv = __shfl_sync(0xffffffffu, wv, wl);
+        if (lane == wl) taken |= 1u << (wi >> 5);
+        if (lane == j) { sel = (int)wi; sel_l = wv; }
+        last = w >> 8;
+    }
+    // exact when no unpicked expert shares the k-th pick's 24-bit key
+    unsigned clash = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; i++)
+        if (!((taken >> i) & 1u) && lane + 32 * i < a.E && (pk[i] >> 8) == last) clash = 1;
+    double m;
+    if (__any_sync(0xffffffffu, clash != 0)) {
+        topk_exact_rounds(a, v, key, lane, sel, sel_l, m);
+    } else {
+        // order the k picks exactly: rank by (logit desc, index asc)
+        int rank = 0;
+        for (int i = 0; i < a.k; i++) {
+            const double vi = __shfl_sync(0xffffffffu, sel_l, i);
+            const int ei = __shfl_sync(0xffffffffu, sel, i);
+            if (lane < a.k && (vi > sel_l || (vi == sel_l && ei < sel))) rank++;
+        }
+        int s2 = sel;
+        double l2 = sel_l;
+        for (int i = 0; i < a.k; i++) {
+            const double vi = __shfl_sync(0xffffffffu, sel_l, i);
+            const int ei = __shfl_sync(0xffffffffu, sel, i);
+            const int ri = __shfl_sync(0xffffffffu, rank, i);
+            if (ri == lane) { s2 = ei; l2 = vi; }
+        }
+        sel = s2;
+        sel_l = l2;
+        m = __shfl_sync(0xffffffffu, sel_l, 0);
     }
     if (lane == 0) fused_trace(a, kTrTopkSelected);
     float w = 0.f;
@@ -552,6 +615,8 @@ __device__ __forceinline__ void fused_producer(const FusedArgs& a, uint8_t* stag
 // ------------------------------------------------------------- consumers --
 struct ConsumerShared {
     unsigned long long rsum[kFusedMaxStages][kRouterRows];   // exact router row sums
+    double rscale[kRouterRows];          // row scales / biases of the first router item
+    double rbias[kRouterRows];
     int item_cnt[kFusedMaxStages];       // warps done with the stage's item
     int down_flag;                       // all gate/up items of the launch done
     int gu_done_local;                   // this CTA's finished gate/up items
@@ -562,11 +627,22 @@ struct ConsumerShared {
     __half h_rows[kMaxDownItems * 8];    // residual rows of this CTA's down items
 };
 
+__device__ __forceinline__ FusedDesc fused_read_desc(const FusedDesc* p) {
+    FusedDesc d;
+    const uint32_t ds = smem_u32(p);
+    const uint4 d0 = lds128(ds);
+    const uint4 d1 = lds128(ds + 16);
+    d.type = (int)d0.x; d.e_slot = (int)d0.y; d.blk = (int)d0.z; d.rows = (int)d0.w;
+    d.w = __uint_as_float(d1.x); d.item = (int)d1.y;
+    d.pad[0] = d.pad[1] = 0;
+    return d;
+}
+
 template <int MAXC, int MAXD>
 __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* stages, FusedDesc* desc,
                                                 uint64_t* full, uint64_t* empty, __half* xs,
                                                 int8_t* xl, float* red, uint32_t* glimb,
-                                                ConsumerShared* cs) {
+                                                uint8_t* hl, uint64_t* hl_bar, ConsumerShared* cs) {
     const int tid = threadIdx.x;                 // 0..255
     const int warp = tid >> 5, lane = tid & 31;
     const int H = a.H;
@@ -577,6 +653,13 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
     // the wait below), then this layer's input (waits for the previous layer)
     unsigned long long ent = 0;
     if (tid == 0) ent = atomicAdd(&a.sync->entries, 1ull);
+    // this CTA's first router item's row scales and biases (weights: they do
+    // not depend on the previous layer)
+    if (tid < kRouterRows && (int)blockIdx.x < a.NR) {
+        const int e = kRouterRows * (int)blockIdx.x + tid;
+        cs->rscale[tid] = e < a.E ? (double)__half2float(a.rscale[e]) : 0.0;
+        cs->rbias[tid] = (e < a.E && a.rbias) ? (double)a.rbias[e] : 0.0;
+    }
     griddep_wait();
     constexpr int kHPer = 16;                    // h values per thread (H <= 4096)
     if (a.prenorm) {
@@ -688,66 +771,6 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
     }
     if (tid == 0) fused_trace(a, kTrProRouterLimbs);
 
-    // ---- x limbs: one thread per 8-column word builds the shared table
-    // (group max over the 8 words of its 64-column group by shuffles); lane
-    // then owns chunks lane + 32 i of every row
-    const int nch = H / 32;
-    const uint32_t xs_s = smem_u32(xs);
-    const uint32_t gl_s = smem_u32(glimb);
-    if (a.NSG + a.NRG > 0) {
-        for (int base = 0; base < H / 8; base += nthr) {
-            const int wd = base + tid;
-            const bool valid = wd < H / 8;
-            float v[8];
-            float m = 0.f, sx = 0.f;
-            {
-                const uint4 q = valid ? lds128(xs_s + 16 * wd) : make_uint4(0, 0, 0, 0);
-                const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                for (int u = 0; u < 4; u++) {
-                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&qq[u]));
-                    v[2 * u] = f.x;
-                    v[2 * u + 1] = f.y;
-                    m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
-                    sx += f.x + f.y;
-                }
-            }
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-            sx += __shfl_xor_sync(0xffffffffu, sx, 1);
-            sx += __shfl_xor_sync(0xffffffffu, sx, 2);
-            const int E = block_exp(m);
-            uint32_t eh, oh, el, ol;
-            word_limbs(v, E, eh, oh, el, ol);
-            if (valid) {
-                const int c = wd >> 2, j = wd & 3;
-                uint32_t* dst = glimb + (size_t)c * kLimbWords;
-                dst[j] = eh; dst[4 + j] = oh; dst[8 + j] = el; dst[12 + j] = ol;
-                if (j == 0) {
-                    dst[16] = __float_as_uint(exp2_int(E - 15));
-                    dst[17] = __float_as_uint(sx);
-                }
-            }
-        }
-        named_bar(1, nthr);
-    }
-    XLimbs gl[MAXC];
-#pragma unroll
-    for (int i = 0; i < MAXC; i++) {
-        const int c = lane + 32 * i;
-        const uint32_t src = gl_s + 4u * (uint32_t)((c < nch ? c : 0) * kLimbWords);
-        const uint4 a0 = lds128(src), a1 = lds128(src + 16), a2 = lds128(src + 32),
-                    a3 = lds128(src + 48);
-        gl[i].eh[0] = a0.x; gl[i].eh[1] = a0.y; gl[i].eh[2] = a0.z; gl[i].eh[3] = a0.w;
-        gl[i].oh[0] = a1.x; gl[i].oh[1] = a1.y; gl[i].oh[2] = a1.z; gl[i].oh[3] = a1.w;
-        gl[i].el[0] = a2.x; gl[i].el[1] = a2.y; gl[i].el[2] = a2.z; gl[i].el[3] = a2.w;
-        gl[i].ol[0] = a3.x; gl[i].ol[1] = a3.y; gl[i].ol[2] = a3.z; gl[i].ol[3] = a3.w;
-        gl[i].fexp = __uint_as_float(lds32(src + 64));
-        gl[i].sx = __uint_as_float(lds32(src + 68));
-    }
-    if (tid == 0) fused_trace(a, kTrProTable);
-    fused_trace(a, kTrPrologue);
 
     // ---- h limbs for the down rows: lane owns chunk tid + 256 j of the
     // concatenated intermediate (routed 0..k-1, then shared), loaded once
@@ -764,17 +787,13 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
 
     int stage = 0;
     uint32_t phase = 0;
-    for (;;) {
-        if (!fused_wait_bar(&full[stage], phase, a.status)) break;
-        FusedDesc d;
-        {
-            const uint32_t ds = smem_u32(desc + stage);
-            const uint4 d0 = lds128(ds);
-            const uint4 d1 = lds128(ds + 16);
-            d.type = (int)d0.x; d.e_slot = (int)d0.y; d.blk = (int)d0.z; d.rows = (int)d0.w;
-            d.w = __uint_as_float(d1.x); d.item = (int)d1.y;
-        }
-        if (d.type < 0) break;
+    // ---- router items first: a CTA's router items are its first items, and
+    // the routing they lead to is the critical path of the launch
+    bool aborted = false;
+    const int n_router = (int)blockIdx.x < a.NR ? (a.NR - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    for (int ri = 0; ri < n_router; ri++) {
+        if (!fused_wait_bar(&full[stage], phase, a.status)) { aborted = true; break; }
+        const FusedDesc d = fused_read_desc(desc + stage);
         const uint32_t st_s = smem_u32(stages) + (uint32_t)stage * a.stage_bytes;
         float* rs = red + (size_t)stage * 64;
         if (first) {
@@ -782,17 +801,22 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
             first = false;
         }
         if (warp == 0 && lane == 0) fused_trace_item(a, n_done, 1, d.type);
-        if (d.type == 0) {
+        {
             // -------- router rows: warp w -> row w / 4 of the item, quarter
             // w % 4 of its columns; exact partial sums meet in shared memory
             cnt_r++;
             const int row = warp >> 2, qt = warp & 3;
-            // lane r holds row r's scale and bias, fetched now for whichever
-            // warp turns out to finish the item
+            // lane r holds row r's scale and bias for whichever warp turns
+            // out to finish the item (the first item's were loaded at entry)
             double scale = 0.0, bias = 0.0;
             if (lane < d.rows) {
-                scale = (double)__half2float(a.rscale[kRouterRows * d.blk + lane]);
-                if (a.rbias) bias = (double)a.rbias[kRouterRows * d.blk + lane];
+                if (ri == 0) {
+                    scale = cs->rscale[lane];
+                    bias = cs->rbias[lane];
+                } else {
+                    scale = (double)__half2float(a.rscale[kRouterRows * d.blk + lane]);
+                    if (a.rbias) bias = (double)a.rbias[kRouterRows * d.blk + lane];
+                }
             }
             if (row < d.rows) {
                 int acc[kRouterMaxLimbs];
@@ -860,7 +884,88 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
                     if (lane == 0) fused_trace(a, kTrTopk);
                 }
             }
-        } else if (d.type == 1) {
+        }
+        __syncwarp();
+        if (warp == 0 && lane == 0) fused_trace_item(a, n_done, 2, d.type);
+        n_done++;
+        if (lane == 0) mbar_arrive(&empty[stage]);
+        if (++stage == a.n_stages) { stage = 0; phase ^= 1u; }
+    }
+
+    // ---- x limbs: one thread per 8-column word builds the shared table
+    // (group max over the 8 words of its 64-column group by shuffles); lane
+    // then owns chunks lane + 32 i of every row
+    const int nch = H / 32;
+    const uint32_t xs_s = smem_u32(xs);
+    const uint32_t gl_s = smem_u32(glimb);
+    if (a.NSG + a.NRG > 0) {          // every consumer thread reaches the barrier below
+        for (int base = 0; base < H / 8; base += nthr) {
+            const int wd = base + tid;
+            const bool valid = wd < H / 8;
+            float v[8];
+            float m = 0.f, sx = 0.f;
+            {
+                const uint4 q = valid ? lds128(xs_s + 16 * wd) : make_uint4(0, 0, 0, 0);
+                const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&qq[u]));
+                    v[2 * u] = f.x;
+                    v[2 * u + 1] = f.y;
+                    m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+                    sx += f.x + f.y;
+                }
+            }
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+            sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+            sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+            const int E = block_exp(m);
+            uint32_t eh, oh, el, ol;
+            word_limbs(v, E, eh, oh, el, ol);
+            if (valid) {
+                const int c = wd >> 2, j = wd & 3;
+                uint32_t* dst = glimb + (size_t)c * kLimbWords;
+                dst[j] = eh; dst[4 + j] = oh; dst[8 + j] = el; dst[12 + j] = ol;
+                if (j == 0) {
+                    dst[16] = __float_as_uint(exp2_int(E - 15));
+                    dst[17] = __float_as_uint(sx);
+                }
+            }
+        }
+        named_bar(1, nthr);
+    }
+    XLimbs gl[MAXC];
+#pragma unroll
+    for (int i = 0; i < MAXC; i++) {
+        const int c = lane + 32 * i;
+        const uint32_t src = gl_s + 4u * (uint32_t)((c < nch ? c : 0) * kLimbWords);
+        const uint4 a0 = lds128(src), a1 = lds128(src + 16), a2 = lds128(src + 32),
+                    a3 = lds128(src + 48);
+        gl[i].eh[0] = a0.x; gl[i].eh[1] = a0.y; gl[i].eh[2] = a0.z; gl[i].eh[3] = a0.w;
+        gl[i].oh[0] = a1.x; gl[i].oh[1] = a1.y; gl[i].oh[2] = a1.z; gl[i].oh[3] = a1.w;
+        gl[i].el[0] = a2.x; gl[i].el[1] = a2.y; gl[i].el[2] = a2.z; gl[i].el[3] = a2.w;
+        gl[i].ol[0] = a3.x; gl[i].ol[1] = a3.y; gl[i].ol[2] = a3.z; gl[i].ol[3] = a3.w;
+        gl[i].fexp = __uint_as_float(lds32(src + 64));
+        gl[i].sx = __uint_as_float(lds32(src + 68));
+    }
+    if (tid == 0) fused_trace(a, kTrProTable);
+    fused_trace(a, kTrPrologue);
+
+    // ---- gate/up and down items
+    for (;;) {
+        if (aborted || !fused_wait_bar(&full[stage], phase, a.status)) break;
+        FusedDesc d = fused_read_desc(desc + stage);
+        if (d.type < 0) break;
+        const uint32_t st_s = smem_u32(stages) + (uint32_t)stage * a.stage_bytes;
+        float* rs = red + (size_t)stage * 64;
+        if (first) {
+            if (warp == 0 && lane == 0) fused_trace(a, kTrFirstItem);
+            first = false;
+        }
+        if (warp == 0 && lane == 0) fused_trace_item(a, n_done, 1, d.type);
+        if (d.type == 1) {
             // -------- gate/up rows: warp w -> intermediate indices
             // 16*blk + 2w and + 2w + 1 (gate rows and up rows of both)
             cnt_gu++;
@@ -953,22 +1058,26 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
             // -------- down rows of every expert + combine
             cnt_d++;
             if (!down_ready) {
-                // warp 0 publishes this CTA's gate/up items if not yet done and
-                // polls the global count; the others poll its flag
+                // warp 0 publishes this CTA's gate/up items if not yet done,
+                // waits for all of the launch's, then copies the packed h
+                // table into shared memory with one bulk copy; every warp
+                // waits for that copy
                 bool ok = true;
-                if (lane == 0) {
-                    if (warp == 0) {
-                        if (cnt_gu > 0 && atomicCAS(&cs->gu_pub, 0, 1) == 0)
-                            ok = fused_publish_gu(a, &cs->gu_done_local, cnt_gu);
-                        ok = ok && fused_wait_ge(&a.sync->gu_done, (ep + 1) * ngu, a.status);
-                        if (ok) { *(volatile int*)&cs->down_flag = 1; fused_trace(a, kTrDownReady); }
-                    } else {
-                        ok = fused_wait_smem(&cs->down_flag, 1, a.status);
+                if (warp == 0 && lane == 0) {
+                    if (cnt_gu > 0 && atomicCAS(&cs->gu_pub, 0, 1) == 0)
+                        ok = fused_publish_gu(a, &cs->gu_done_local, cnt_gu);
+                    ok = ok && fused_wait_ge(&a.sync->gu_done, (ep + 1) * ngu, a.status);
+                    if (ok) {
+                        fused_trace(a, kTrDownReady);
+                        fence_proxy_async_global();
+                        const uint32_t bytes = (uint32_t)NC * kDLimbWords * 4;
+                        mbar_arrive_expect_tx(hl_bar, bytes);
+                        bulk_g2s(hl, a.dlimb, bytes, hl_bar);
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                if (!ok) break;
-                fence_acq_rel_gpu();
+                if (!ok || !fused_wait_bar(hl_bar, 0, a.status)) break;
+                const uint32_t hl_s = smem_u32(hl);
 #pragma unroll
                 for (int j = 0; j < MAXD; j++) {
                     const int L = tid + 256 * j;
@@ -978,9 +1087,9 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
                     const int ce = !valid ? 0 : (e < a.k ? L - e * (a.I / 32) : L - kI32);
                     const int Ie = e < a.k ? a.I : a.Is;
                     uint4 t[6];
-                    const uint4* src = reinterpret_cast<const uint4*>(a.dlimb + (size_t)(valid ? L : 0) * kDLimbWords);
+                    const uint32_t src = hl_s + (uint32_t)(valid ? L : 0) * (kDLimbWords * 4);
 #pragma unroll
-                    for (int u = 0; u < 6; u++) t[u] = valid ? __ldcg(src + u) : make_uint4(0, 0, 0, 0);
+                    for (int u = 0; u < 6; u++) t[u] = valid ? lds128(src + 16 * u) : make_uint4(0, 0, 0, 0);
                     dl[j].eh[0] = t[0].x; dl[j].eh[1] = t[0].y; dl[j].eh[2] = t[0].z; dl[j].eh[3] = t[0].w;
                     dl[j].oh[0] = t[1].x; dl[j].oh[1] = t[1].y; dl[j].oh[2] = t[1].z; dl[j].oh[3] = t[1].w;
                     dl[j].el[0] = t[2].x; dl[j].el[1] = t[2].y; dl[j].el[2] = t[2].z; dl[j].el[3] = t[2].w;
@@ -1073,16 +1182,18 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
 // reductions [stages][64] floats, x limb table [H/32][20] words,
 // descriptors, barriers, producer and consumer scalars.
 struct FusedSmemLayout {
-    size_t xs, xl, red, glimb, desc, full, empty, ps, cs, total;
-    __host__ __device__ FusedSmemLayout(int H, int n_stages, int stage_bytes) {
+    size_t xs, xl, red, glimb, hl, desc, full, empty, hlbar, ps, cs, total;
+    __host__ __device__ FusedSmemLayout(int H, int NC, int n_stages, int stage_bytes) {
         size_t off = (size_t)n_stages * stage_bytes;
         xs = off;    off += ((size_t)H * 2 + 127) / 128 * 128;
         xl = off;    off += ((size_t)kRouterMaxLimbs * H + 127) / 128 * 128;
         red = off;   off += (size_t)n_stages * 64 * sizeof(float);
         glimb = off; off += ((size_t)(H / 32) * kLimbWords * 4 + 15) / 16 * 16;
+        hl = off;    off += (size_t)NC * kDLimbWords * 4;
         desc = off;  off += (size_t)n_stages * sizeof(FusedDesc);
         full = off;  off += (size_t)n_stages * 8;
         empty = off; off += (size_t)n_stages * 8;
+        hlbar = off; off += 8;
         ps = off;    off += (sizeof(ProducerShared) + 15) / 16 * 16;
         cs = off;    off += (sizeof(ConsumerShared) + 15) / 16 * 16;
         total = off;
@@ -1092,7 +1203,7 @@ struct FusedSmemLayout {
 template <int MAXC, int MAXD>
 __global__ void __launch_bounds__(kFusedThreads, 1) k_moe_layer_fused(const FusedArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const FusedSmemLayout lay(a.H, a.n_stages, a.stage_bytes);
+    const FusedSmemLayout lay(a.H, (a.k * a.I + a.Is) / 32, a.n_stages, a.stage_bytes);
     uint8_t* stages = smem;
     __half* xs = reinterpret_cast<__half*>(smem + lay.xs);
     int8_t* xl = reinterpret_cast<int8_t*>(smem + lay.xl);
@@ -1101,6 +1212,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_moe_layer_fused(const Fuse
     FusedDesc* desc = reinterpret_cast<FusedDesc*>(smem + lay.desc);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.full);
     uint64_t* empty = reinterpret_cast<uint64_t*>(smem + lay.empty);
+    uint8_t* hl = smem + lay.hl;
+    uint64_t* hl_bar = reinterpret_cast<uint64_t*>(smem + lay.hlbar);
     ProducerShared* ps = reinterpret_cast<ProducerShared*>(smem + lay.ps);
     ConsumerShared* cs = reinterpret_cast<ConsumerShared*>(smem + lay.cs);
 
@@ -1112,6 +1225,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_moe_layer_fused(const Fuse
             cs->item_cnt[s] = 0;
             for (int r = 0; r < kRouterRows; r++) cs->rsum[s][r] = 0;
         }
+        mbar_init(hl_bar, 1);
         cs->down_flag = 0;
         cs->gu_done_local = 0;
         cs->gu_final = -1;
@@ -1127,12 +1241,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_moe_layer_fused(const Fuse
                        threadIdx.x & 31);
         return;
     }
-    fused_consumers<MAXC, MAXD>(a, stages, desc, full, empty, xs, xl, red, glimb, cs);
+    fused_consumers<MAXC, MAXD>(a, stages, desc, full, empty, xs, xl, red, glimb, hl, hl_bar, cs);
 }
 
 // Shared memory bytes besides the stage ring.
-__host__ inline size_t fused_fixed_smem(int H, int n_stages) {
-    return FusedSmemLayout(H, n_stages, 0).total;
+__host__ inline size_t fused_fixed_smem(int H, int NC, int n_stages) {
+    return FusedSmemLayout(H, NC, n_stages, 0).total;
 }
 
 }  // namespace moeq4

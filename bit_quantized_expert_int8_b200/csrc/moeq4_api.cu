@@ -97,6 +97,7 @@ struct moe_ctx {
     bool fused_ok = false;
     uint32_t* dlimb = nullptr;         // packed intermediate of the fused kernel
     int f_stages = 0, f_stage_bytes = 0;
+    int f_regs = 0, f_max_threads = 0;
     unsigned long long* trace = nullptr;   // [n_sms * 16] phase stamps
     bool tracing = false;
     size_t f_smem = 0;
@@ -163,7 +164,7 @@ static cudaError_t setup_fused(moe_ctx* c) {
     stage = (stage + 127) / 128 * 128;
     int ns = 0;
     for (int n = kFusedMaxStages; n >= 2 && ns == 0; n--)
-        if ((size_t)n * stage + fused_fixed_smem(g.hidden, n) <= (size_t)optin) ns = n;
+        if ((size_t)n * stage + fused_fixed_smem(g.hidden, NC, n) <= (size_t)optin) ns = n;
     c->fused_ok = g.hidden <= 4096 && maxc >= 1 && maxc <= 4 && maxd >= 1 && maxd <= 2 &&
                   ns >= 2 && stage < (1u << 20) && c->n_sms > 0;
     if (!c->fused_ok) return cudaSuccess;
@@ -174,9 +175,18 @@ static cudaError_t setup_fused(moe_ctx* c) {
         {k_moe_layer_fused<3, 1>, k_moe_layer_fused<3, 2>},
         {k_moe_layer_fused<4, 1>, k_moe_layer_fused<4, 2>}};
     c->f_kernel = table[maxc - 1][maxd - 1];
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, c->f_kernel);
+    if (e != cudaSuccess) return e;
+    c->f_regs = fa.numRegs;
+    c->f_max_threads = fa.maxThreadsPerBlock;
+    if (fa.maxThreadsPerBlock < kFusedThreads) {    // registers would not fit: use the direct kernels
+        c->fused_ok = false;
+        return cudaSuccess;
+    }
     c->f_stages = ns;
     c->f_stage_bytes = (int)stage;
-    c->f_smem = (size_t)ns * stage + fused_fixed_smem(g.hidden, ns);
+    c->f_smem = (size_t)ns * stage + fused_fixed_smem(g.hidden, NC, ns);
     return cudaFuncSetAttribute(c->f_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)c->f_smem);
 }
@@ -587,6 +597,16 @@ extern "C" int moe_ctx_check(moe_ctx* c, moe_stream_t stream) {
     CK(cudaMemset(c->fsync, 0, 8 * sizeof(FusedSync)));
     for (int m = 0; m < 4; m++) c->fparity[m] = 0;
     return fail(st, "a bounded device wait gave up (status %d); counters reset", st);
+}
+
+extern "C" int moe_ctx_info(moe_ctx* c, char* buf, int len) {
+    if (!c || !buf || len < 1) return fail(MOE_ERR_INVALID_ARG, "moe_ctx_info: bad argument");
+    int n = snprintf(buf, (size_t)len,
+                     "single-token path: %s; sms %d; stages %d x %d B; smem %zu B; "
+                     "registers %d; max threads %d (needs %d)",
+                     c->fused_ok ? "fused" : "direct kernels", c->n_sms, c->f_stages,
+                     c->f_stage_bytes, c->f_smem, c->f_regs, c->f_max_threads, kFusedThreads);
+    return n < 0 ? fail(MOE_ERR_INVALID_ARG, "moe_ctx_info: format") : MOE_OK;
 }
 
 extern "C" int moe_ctx_trace(moe_ctx* c, int enable, unsigned long long* host_out,

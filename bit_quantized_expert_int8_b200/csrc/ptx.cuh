@@ -113,6 +113,12 @@ __device__ __forceinline__ uint16_t lds16(uint32_t addr) {
     return v;
 }
 
+// Orders this thread's view of global data written through the generic
+// proxy (then acquired) before its later bulk asynchronous copies read it.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Named barrier among the consumer warps only.
 __device__ __forceinline__ void named_bar(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");

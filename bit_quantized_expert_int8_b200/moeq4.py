@@ -27,7 +27,7 @@ MOE_ERR_CACHE_STATE = -6
 MOE_PRENORM = 1
 MOE_MAX_SLOTS = 32
 
-EXPORTS = ("moe_ctx_create", "moe_ctx_destroy", "moe_ctx_check", "moe_ctx_trace",
+EXPORTS = ("moe_ctx_create", "moe_ctx_destroy", "moe_ctx_check", "moe_ctx_trace", "moe_ctx_info",
            "moe_last_error", "moe_blob_bytes",
            "moe_router_topk", "moe_expert_ffn_q4", "moe_combine", "moe_lfu_init",
            "moe_cache_lookup_lfu", "moe_layer_decode", "moe_stack_decode")
@@ -88,6 +88,7 @@ def load() -> ctypes.CDLL:
         "moe_ctx_destroy": ([P], i32),
         "moe_ctx_check": ([P, P], i32),
         "moe_ctx_trace": ([P, i32, P, i32], i32),
+        "moe_ctx_info": ([P, ctypes.c_char_p, i32], i32),
         "moe_last_error": ([], ctypes.c_char_p),
         "moe_blob_bytes": ([i32, i32], ctypes.c_size_t),
         "moe_router_topk": ([P, P, P, P, P, i32, P, P, P, P], i32),
@@ -165,6 +166,14 @@ def moe_ctx_check(ctx, stream=None):
     """Synchronise and raise MoeError(MOE_ERR_TIMEOUT) if a bounded device
     wait of this context gave up since the last check."""
     _check(load().moe_ctx_check(ctx.handle, _stream(stream)))
+
+
+def moe_ctx_info(ctx) -> str:
+    """moe_ctx_info: which kernels serve single-token layers, and their
+    shared memory and registers."""
+    buf = ctypes.create_string_buffer(512)
+    _check(load().moe_ctx_info(ctx.handle, buf, 512))
+    return buf.value.decode()
 
 
 def moe_ctx_trace(ctx, enable=-1, read=False):

@@ -103,6 +103,12 @@ int moe_ctx_destroy(moe_ctx *ctx);
  * context's counters reset so that it can be used again) or MOE_OK. */
 int moe_ctx_check(moe_ctx *ctx, moe_stream_t stream);
 
+/* One line describing the context: which kernels serve single-token layers
+ * (the fused layer kernel, or the direct kernels when the shape or the device
+ * does not fit it), its shared-memory ring and register use.  Writes at most
+ * len bytes (NUL-terminated) into buf (host). */
+int moe_ctx_info(moe_ctx *ctx, char *buf, int len);
+
 /* Tracing of the single-token layer kernel.  enable = 1 makes later launches
  * record, per CTA, 160 words: globaltimer stamps (ns) of kernel entry, end of
  * the input prologue, first item, routing known, down phase ready, consumer
