@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -680,5 +681,82 @@ extern "C" int moe_stack_decode(moe_ctx* c, const MoeLayer* layers, int n_layers
     }
     CK(cudaMemsetAsync(c->cursor, 0, sizeof(int), stream));
     for (int t = 0; t < T; t++) CK(cudaGraphLaunch(c->stack_exec, stream));
+    return MOE_OK;
+}
+
+// ------------------------------------------------- router, no allocation --
+// moe_router_topk_noalloc: the router above without a context.  Its scratch
+// (the fp64 logits of every token and one completion counter per token) lives
+// in this file-scope device array, which every GPU that loads the library
+// holds until the process exits.  In host code the name is only a stand-in
+// for the symbol; the device address comes from cudaGetSymbolAddress.
+constexpr int kNoAllocMaxLogits = 8192;                  // T * n_experts
+constexpr int kNoAllocMaxTokens = 256;
+constexpr int kNoAllocMaxHidden = 6144;                  // x*2^24 as int64 in 48 KiB
+constexpr size_t kNoAllocCounterOff = (size_t)kNoAllocMaxLogits * sizeof(double);
+constexpr size_t kNoAllocScratchBytes = kNoAllocCounterOff + kNoAllocMaxTokens * sizeof(int);
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_router_scratch[kNoAllocScratchBytes];
+
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_dev_ptr[kNoAllocMaxDevices];      // per device ordinal
+
+// Device address of the scratch array on the current device, looked up once
+// per device (with that device current) and remembered.
+static int noalloc_scratch(unsigned char** out) {
+    int dev = -1;
+    CK(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kNoAllocMaxDevices)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_router_topk_noalloc: device %d above %d", dev,
+                    kNoAllocMaxDevices - 1);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_dev_ptr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_router_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(MOE_ERR_CUDA, "moe_router_topk_noalloc: cudaGetSymbolAddress: %s",
+                        cudaGetErrorString(e));
+        g_noalloc_dev_ptr[dev] = p;
+    }
+    *out = static_cast<unsigned char*>(g_noalloc_dev_ptr[dev]);
+    return MOE_OK;
+}
+
+extern "C" int moe_router_topk_noalloc(int n_experts, int hidden, int top_k, int renorm,
+                                       const int8_t* Wr, const moe_half* row_scale,
+                                       const float* bias, const moe_half* x, int T,
+                                       int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+    if (!Wr || !row_scale || !x || !topk_idx || !topk_w)
+        return fail(MOE_ERR_INVALID_ARG, "moe_router_topk_noalloc: NULL argument");
+    if (top_k < 1 || top_k > MOE_MAX_TOPK || n_experts < top_k || n_experts > MOE_MAX_EXPERTS)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                    "moe_router_topk_noalloc: need 1 <= top_k <= 8, top_k <= n_experts <= 256");
+    if (hidden <= 0 || hidden % MOE_GROUP || hidden > kNoAllocMaxHidden)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                    "moe_router_topk_noalloc: hidden=%d must be a positive multiple of 64 <= %d",
+                    hidden, kNoAllocMaxHidden);
+    if (renorm != 0 && renorm != 1)
+        return fail(MOE_ERR_INVALID_ARG, "moe_router_topk_noalloc: renorm must be 0 or 1");
+    if (T < 1) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_router_topk_noalloc: T must be >= 1");
+    if (T > kNoAllocMaxTokens || (long long)T * n_experts > kNoAllocMaxLogits)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                    "moe_router_topk_noalloc: T=%d with n_experts=%d exceeds the static scratch "
+                    "(T <= %d and T * n_experts <= %d)",
+                    T, n_experts, kNoAllocMaxTokens, kNoAllocMaxLogits);
+    if (!aligned16(Wr) || !aligned16(row_scale) || !aligned16(x) || !aligned4(topk_idx) ||
+        !aligned4(topk_w) || (bias && !aligned4(bias)))
+        return fail(MOE_ERR_ALIGNMENT, "moe_router_topk_noalloc: misaligned pointer");
+    unsigned char* scratch = nullptr;
+    TRY(noalloc_scratch(&scratch));
+    double* logits = reinterpret_cast<double*>(scratch);
+    int* done = reinterpret_cast<int*>(scratch + kNoAllocCounterOff);
+    // the array keeps the previous call's contents: the counters start at 0
+    CK(cudaMemsetAsync(done, 0, (size_t)T * sizeof(int), stream));
+    dim3 grid((n_experts + kRouterWarps - 1) / kRouterWarps, T);
+    k_router<<<grid, 256, (size_t)hidden * sizeof(long long), stream>>>(
+        Wr, reinterpret_cast<const __half*>(row_scale), bias, reinterpret_cast<const __half*>(x),
+        n_experts, hidden, top_k, renorm, logits, done, topk_idx, topk_w);
+    CKL();
     return MOE_OK;
 }

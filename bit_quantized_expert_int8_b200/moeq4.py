@@ -30,7 +30,8 @@ MOE_MAX_SLOTS = 32
 EXPORTS = ("moe_ctx_create", "moe_ctx_destroy", "moe_ctx_check", "moe_ctx_trace", "moe_ctx_info",
            "moe_last_error", "moe_blob_bytes",
            "moe_router_topk", "moe_expert_ffn_q4", "moe_combine", "moe_lfu_init",
-           "moe_cache_lookup_lfu", "moe_layer_decode", "moe_stack_decode")
+           "moe_cache_lookup_lfu", "moe_layer_decode", "moe_stack_decode",
+           "moe_router_topk_noalloc")
 
 
 class MoeError(RuntimeError):
@@ -99,6 +100,7 @@ def load() -> ctypes.CDLL:
         "moe_layer_decode": ([P, ctypes.POINTER(CMoeLayer), P, i32,
                               ctypes.POINTER(CMoeLayerOut), i32, P, P], i32),
         "moe_stack_decode": ([P, P, i32, P, i32, P, P], i32),
+        "moe_router_topk_noalloc": ([i32, i32, i32, i32, P, P, P, P, i32, P, P, P], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -193,6 +195,15 @@ def moe_ctx_trace(ctx, enable=-1, read=False):
 def moe_router_topk(ctx, Wr, row_scale, bias, x, T, topk_idx, topk_w, logits=None, stream=None):
     _check(load().moe_router_topk(ctx.handle, _ptr(Wr), _ptr(row_scale), _ptr(bias), _ptr(x), T,
                                   _ptr(topk_idx), _ptr(topk_w), _ptr(logits), _stream(stream)))
+
+
+def moe_router_topk_noalloc(n_experts, hidden, top_k, renorm, Wr, row_scale, bias, x, T,
+                            topk_idx, topk_w, stream=None):
+    """Router without a context for callers that cannot allocate device
+    memory; its scratch is a static device array (limits in include/moeq4.h)."""
+    _check(load().moe_router_topk_noalloc(n_experts, hidden, top_k, renorm, _ptr(Wr),
+                                          _ptr(row_scale), _ptr(bias), _ptr(x), T,
+                                          _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
 
 
 def make_pairs(entries, device="cuda"):

@@ -165,6 +165,32 @@ int moe_router_topk(moe_ctx *ctx, const int8_t *Wr, const moe_half *row_scale,
                     int32_t *topk_idx, float *topk_w, double *logits,
                     moe_stream_t stream);
 
+/* ------------------------------------------- router, no allocation ----
+ * The router above (same arithmetic, same outputs) for callers that cannot
+ * allocate device memory: code running under another runtime's allocator or
+ * a fixed device-memory budget, where cudaMalloc would bypass the owner's
+ * accounting, and latency-bound loops where cudaMalloc/cudaFree would stall
+ * on their implicit device synchronisation.  It takes no moe_ctx (creating
+ * one allocates a workspace) and itself calls no cudaMalloc, cudaFree or
+ * other allocating routine.  The pages describe no such entry point.
+ *   n_experts, hidden, top_k, renorm  as in MoeConfig
+ *   Wr, row_scale, bias, x, topk_idx, topk_w  as for moe_router_topk
+ *   (the logits are not returned).
+ * Scratch: the logits and per-token counters live in one static device
+ * array of 66,560 bytes that every GPU loading this library holds until
+ * exit.  Limits: T <= 256, T * n_experts <= 8192, hidden a multiple of 64
+ * and <= 6144; larger requests return MOE_ERR_UNSUPPORTED_SHAPE before any
+ * CUDA call.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture.  Every call on a device shares the one
+ * array: calls whose executions overlap on the GPU (other streams, other
+ * host threads) race on it and must be serialised by the caller. */
+int moe_router_topk_noalloc(int n_experts, int hidden, int top_k, int renorm,
+                            const int8_t *Wr, const moe_half *row_scale,
+                            const float *bias, const moe_half *x, int T,
+                            int32_t *topk_idx, float *topk_w,
+                            moe_stream_t stream);
+
 /* ----------------------------------------------------- expert FFN ----
  * Grouped expert FFN over n_pairs (expert, token) pairs: for pair p,
  *   g = Wg x, u = Wu x, h = GELU(g) * u, y[p] = Wd h,
