@@ -338,73 +338,93 @@ __device__ __forceinline__ void topk_exact_rounds(const FusedArgs& a, const doub
 
 // Top-k of logits[0..E), largest first, ties to the lower index, then the
 // softmax weights of the selected experts, published as the launch's tagged
-// routing record and to the caller's outputs.  Fast path: one max-reduction
-// per round on (24-bit order key << 8 | 255 - index); the 24-bit key is a
-// monotone function of the logit, so every expert whose key beats the k-th
-// pick's key is in the exact top-k and every expert below it is out; when no
-// other expert shares the k-th key the picked set is exact, and its order is
-// then settled by exact fp64 comparisons.  Otherwise the exact rounds run.
+// routing record and to the caller's outputs.
+//
+// Fast path (E <= 128): each lane sorts its four experts by a packed word
+// (24-bit order key << 8 | 255 - index), and each round takes the maximum of
+// the lane heads with one reduction, the winning lane popping its head.  The
+// 24-bit key is a monotone function of the logit, so the picked set is the
+// exact top-k unless an unpicked expert shares the k-th pick's key, and the
+// pick order is exact unless two picks share a key; those cases are settled
+// by exact fp64 comparisons (a rank sort of the k picks, or the exact rounds
+// over all experts).
 __device__ __forceinline__ void fused_topk_publish(const FusedArgs& a, unsigned long long epoch,
                                                    int lane) {
     constexpr int kPer = MOE_MAX_EXPERTS / 32;
-    double v[kPer];
-    unsigned long long key[kPer];
-    unsigned pk[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; i++) {
-        const int e = lane + 32 * i;
-        v[i] = e < a.E ? __ldcg(a.logits + e) : 0.0;
-        key[i] = e < a.E ? order_key(v[i]) : 0ull;      // 0 sorts below every logit
-        pk[i] = e < a.E ? ((unsigned)(key[i] >> 40) << 8) | (unsigned)(255 - e) : 0u;
-    }
-    if (lane == 0) fused_trace(a, kTrTopkLoaded);
-    unsigned taken = 0, last = 0;
     int sel = 0;
-    double sel_l = 0.0;
-    for (int j = 0; j < a.k; j++) {
-        unsigned best = 0;
+    double sel_l = 0.0, m = 0.0;
+    bool exact_rounds = a.E > 128;
+    if (!exact_rounds) {
+        unsigned pk[4];
+        double vv[4];
 #pragma unroll
-        for (int i = 0; i < kPer; i++)
-            if (!((taken >> i) & 1u) && pk[i] > best) best = pk[i];
-        const unsigned w = __reduce_max_sync(0xffffffffu, best);
-        const unsigned wi = 255u - (w & 255u);
-        const int wl = (int)(wi & 31u);
-        double wv = 0.0;
-#pragma unroll
-        for (int i = 0; i < kPer; i++)
-            if ((unsigned)(lane + 32 * i) == wi) wv = v[i];
-        wv = __shfl_sync(0xffffffffu, wv, wl);
-        if (lane == wl) taken |= 1u << (wi >> 5);
-        if (lane == j) { sel = (int)wi; sel_l = wv; }
-        last = w >> 8;
+        for (int i = 0; i < 4; i++) {
+            const int e = lane + 32 * i;
+            vv[i] = e < a.E ? __ldcg(a.logits + e) : 0.0;
+            pk[i] = e < a.E ? ((unsigned)(order_key(vv[i]) >> 40) << 8) | (unsigned)(255 - e) : 0u;
+        }
+        if (lane == 0) fused_trace(a, kTrTopkLoaded);
+        // sorting network, descending: (0,1) (2,3) (0,2) (1,3) (1,2)
+#define MOEQ4_CSWAP(i, j)                                                  \
+        if (pk[j] > pk[i]) {                                               \
+            const unsigned tk = pk[i]; pk[i] = pk[j]; pk[j] = tk;          \
+            const double tv = vv[i]; vv[i] = vv[j]; vv[j] = tv;            \
+        }
+        MOEQ4_CSWAP(0, 1) MOEQ4_CSWAP(2, 3) MOEQ4_CSWAP(0, 2) MOEQ4_CSWAP(1, 3) MOEQ4_CSWAP(1, 2)
+#undef MOEQ4_CSWAP
+        unsigned mk = 0, last = 0;
+        for (int j = 0; j < a.k; j++) {
+            const unsigned w = __reduce_max_sync(0xffffffffu, pk[0]);
+            const int e = 255 - (int)(w & 255u);
+            const int wl = e & 31;
+            const double wv = __shfl_sync(0xffffffffu, vv[0], wl);
+            if (lane == j) { sel = e; sel_l = wv; mk = w; }
+            if (lane == wl) {
+                pk[0] = pk[1]; pk[1] = pk[2]; pk[2] = pk[3]; pk[3] = 0u;
+                vv[0] = vv[1]; vv[1] = vv[2]; vv[2] = vv[3];
+            }
+            last = w >> 8;
+        }
+        // a lane's head is its largest unpicked expert
+        exact_rounds = __any_sync(0xffffffffu, pk[0] != 0u && (pk[0] >> 8) == last);
+        if (!exact_rounds) {
+            const unsigned nx = __shfl_down_sync(0xffffffffu, mk, 1);
+            if (__any_sync(0xffffffffu, lane + 1 < a.k && (mk >> 8) == (nx >> 8))) {
+                // order the k picks exactly: rank by (logit desc, index asc)
+                int rank = 0;
+                for (int i = 0; i < a.k; i++) {
+                    const double vi = __shfl_sync(0xffffffffu, sel_l, i);
+                    const int ei = __shfl_sync(0xffffffffu, sel, i);
+                    if (lane < a.k && (vi > sel_l || (vi == sel_l && ei < sel))) rank++;
+                }
+                int s2 = sel;
+                double l2 = sel_l;
+                for (int i = 0; i < a.k; i++) {
+                    const double vi = __shfl_sync(0xffffffffu, sel_l, i);
+                    const int ei = __shfl_sync(0xffffffffu, sel, i);
+                    const int ri = __shfl_sync(0xffffffffu, rank, i);
+                    if (ri == lane) { s2 = ei; l2 = vi; }
+                }
+                sel = s2;
+                sel_l = l2;
+            }
+            m = __shfl_sync(0xffffffffu, sel_l, 0);
+        }
     }
-    // exact when no unpicked expert shares the k-th pick's 24-bit key
-    unsigned clash = 0;
+    double v[kPer];
+    if (exact_rounds || !a.renorm) {
 #pragma unroll
-    for (int i = 0; i < kPer; i++)
-        if (!((taken >> i) & 1u) && lane + 32 * i < a.E && (pk[i] >> 8) == last) clash = 1;
-    double m;
-    if (__any_sync(0xffffffffu, clash != 0)) {
+        for (int i = 0; i < kPer; i++) {
+            const int e = lane + 32 * i;
+            v[i] = e < a.E ? __ldcg(a.logits + e) : 0.0;
+        }
+    }
+    if (exact_rounds) {
+        unsigned long long key[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; i++)
+            key[i] = lane + 32 * i < a.E ? order_key(v[i]) : 0ull;   // 0 sorts below every logit
         topk_exact_rounds(a, v, key, lane, sel, sel_l, m);
-    } else {
-        // order the k picks exactly: rank by (logit desc, index asc)
-        int rank = 0;
-        for (int i = 0; i < a.k; i++) {
-            const double vi = __shfl_sync(0xffffffffu, sel_l, i);
-            const int ei = __shfl_sync(0xffffffffu, sel, i);
-            if (lane < a.k && (vi > sel_l || (vi == sel_l && ei < sel))) rank++;
-        }
-        int s2 = sel;
-        double l2 = sel_l;
-        for (int i = 0; i < a.k; i++) {
-            const double vi = __shfl_sync(0xffffffffu, sel_l, i);
-            const int ei = __shfl_sync(0xffffffffu, sel, i);
-            const int ri = __shfl_sync(0xffffffffu, rank, i);
-            if (ri == lane) { s2 = ei; l2 = vi; }
-        }
-        sel = s2;
-        sel_l = l2;
-        m = __shfl_sync(0xffffffffu, sel_l, 0);
     }
     if (lane == 0) fused_trace(a, kTrTopkSelected);
     float w = 0.f;

@@ -53,6 +53,48 @@ def test_fused_layer_parity(cfg, bias):
         assert_y_close(y[0].cpu().numpy(), ref["y"], f"{cfg} token {s}")
 
 
+@pytest.mark.parametrize("cfg,boundary_tie", [(RAGGED, False), (WIDE, False), (LAYER, True)])
+def test_fused_router_ties_and_near_ties(cfg, boundary_tie):
+    """Crafted router rows: an exact tie among the picks, two logits that
+    differ only far below the top-k's coarse key (the larger one has the
+    higher index; with k = 3 they compete for the last place), and, when
+    boundary_tie, an exact tie across the k-th place."""
+    L = make_layer(cfg, seed=9)
+    x = synth.tokens(1, cfg.H, seed=10, device=DEV)
+    sgn = torch.sign(x[0].float()).to(torch.int8)
+    xa = x[0].float().abs()
+    c_small = int(torch.where(xa > 0, xa, torch.full_like(xa, 1e9)).argmin())
+    Wr = L["router_w"].clone()
+    sc = L["router_scale"].clone()
+    rows_a = [3, 11]                                   # exact tie, value 100
+    rows_d = [5, 9]                                    # near tie, value 80 (row 9 larger)
+    n_b = max(0, cfg.k - 4 + (1 if boundary_tie else 0))
+    rows_b = list(range(12, 12 + n_b))                 # exact tie, value 50
+    for r in rows_a:
+        Wr[r] = sgn * 100
+    for r in rows_d:
+        Wr[r] = sgn * 80
+    Wr[9, c_small] = sgn[c_small] * 81
+    for r in rows_b:
+        Wr[r] = sgn * 50
+    for r in rows_a + rows_d + rows_b:
+        sc[r] = sc[0]
+    L2 = dict(L, router_w=Wr, router_scale=sc)
+    ctx = moeq4.Context(cfg, 1)
+    lay = moeq4.Layer.from_dict(L2)
+    y = torch.empty((1, cfg.H), device=DEV)
+    idx = torch.empty((1, cfg.k), dtype=torch.int32, device=DEV)
+    w = torch.empty((1, cfg.k), device=DEV)
+    moeq4.moe_layer_decode(ctx, lay, x, 1, y, idx, w)
+    moeq4.moe_ctx_check(ctx)
+    ref = oracle.moe_layer(cfg, np_layer(L2), np_of(x)[0])
+    expect = (rows_a + [9, 5] + rows_b)[:cfg.k]
+    assert ref["idx"].tolist() == expect
+    assert idx[0].cpu().tolist() == expect
+    np.testing.assert_allclose(w[0].cpu().numpy(), ref["w"], rtol=2e-6, atol=1e-7)
+    assert_y_close(y[0].cpu().numpy(), ref["y"], f"{cfg} ties")
+
+
 def test_fused_prenorm_single_token():
     cfg = LAYER
     L = make_layer(cfg, seed=6, bias_std=1.5)
