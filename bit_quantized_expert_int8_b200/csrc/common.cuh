@@ -11,18 +11,45 @@ namespace moeq4 {
 
 constexpr int kGroup = 64;     // weights per quantisation group
 
-// Byte offsets of the six sections of an expert blob (layout in moeq4.h).
+// Tiled expert blob (layout in moeq4.h): I/16 gate/up tiles of 18 H bytes
+// (gate codes [16][H/8] u32, up codes [16][H/8], gate scales [16][H/64]
+// fp16, up scales, gate biases, up biases), then H/16 down tiles of 9 I
+// bytes (codes [16][I/8] u32, scales [16][I/64] fp16, biases).  Byte offsets
+// of one row's codes, scales and biases.
 struct BlobLayout {
-    size_t gu_q, gu_s, gu_b, dn_q, dn_s, dn_b, bytes;
-    __host__ __device__ BlobLayout(int H, int I) {
-        size_t rows = 2 * (size_t)I;
-        gu_q = 0;
-        gu_s = gu_q + rows * (size_t)H / 2;
-        gu_b = gu_s + rows * (size_t)(H / kGroup) * 2;
-        dn_q = gu_b + rows * (size_t)(H / kGroup) * 2;
-        dn_s = dn_q + (size_t)H * (size_t)I / 2;
-        dn_b = dn_s + (size_t)H * (size_t)(I / kGroup) * 2;
-        bytes = dn_b + (size_t)H * (size_t)(I / kGroup) * 2;
+    int H, I;
+    size_t gu_tile, dn_base, dn_tile, bytes;
+    __host__ __device__ BlobLayout(int H_, int I_) : H(H_), I(I_) {
+        gu_tile = 18 * (size_t)H;
+        dn_base = (size_t)(I / 16) * gu_tile;
+        dn_tile = 9 * (size_t)I;
+        bytes = dn_base + (size_t)(H / 16) * dn_tile;
+    }
+    // row r of the gate/up matrix: gate rows 0..I-1, up rows I..2I-1
+    __host__ __device__ size_t gu_row(int r) const {      // 16 * up + position in the tile
+        const int up = r >= I ? 1 : 0, i = r - up * I;
+        return (size_t)(16 * up + i % 16);
+    }
+    __host__ __device__ size_t gu_base(int r) const {
+        const int i = r >= I ? r - I : r;
+        return (size_t)(i / 16) * gu_tile;
+    }
+    __host__ __device__ size_t gu_codes(int r) const { return gu_base(r) + gu_row(r) * (H / 2); }
+    __host__ __device__ size_t gu_scales(int r) const {
+        return gu_base(r) + 16 * (size_t)H + gu_row(r) * (H / 32);
+    }
+    __host__ __device__ size_t gu_biases(int r) const {
+        return gu_base(r) + 17 * (size_t)H + gu_row(r) * (H / 32);
+    }
+    // row r of the down matrix
+    __host__ __device__ size_t dn_codes(int r) const {
+        return dn_base + (size_t)(r / 16) * dn_tile + (size_t)(r % 16) * (I / 2);
+    }
+    __host__ __device__ size_t dn_scales(int r) const {
+        return dn_base + (size_t)(r / 16) * dn_tile + 8 * (size_t)I + (size_t)(r % 16) * (I / 32);
+    }
+    __host__ __device__ size_t dn_biases(int r) const {
+        return dn_base + (size_t)(r / 16) * dn_tile + 17 * (size_t)I / 2 + (size_t)(r % 16) * (I / 32);
     }
 };
 

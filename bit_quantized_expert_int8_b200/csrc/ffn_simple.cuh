@@ -64,12 +64,16 @@ k_ffn_gateup_simple(const MoeFfnPair* __restrict__ pairs, const __half* __restri
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int i = blockIdx.x * 8 + warp;
     if (i >= I) return;
-    BlobLayout L(H, I);
+    const BlobLayout L(H, I);
     const uint8_t* blob = static_cast<const uint8_t*>(pr.blob);
-    const __half* s = reinterpret_cast<const __half*>(blob + L.gu_s);
-    const __half* b = reinterpret_cast<const __half*>(blob + L.gu_b);
-    float g = q4_row_dot_warp(blob + L.gu_q, s, b, H, i, xs, lane);
-    float u = q4_row_dot_warp(blob + L.gu_q, s, b, H, I + i, xs, lane);
+    const float g = q4_row_dot_warp(blob + L.gu_codes(i),
+                                    reinterpret_cast<const __half*>(blob + L.gu_scales(i)),
+                                    reinterpret_cast<const __half*>(blob + L.gu_biases(i)), H, 0,
+                                    xs, lane);
+    const float u = q4_row_dot_warp(blob + L.gu_codes(I + i),
+                                    reinterpret_cast<const __half*>(blob + L.gu_scales(I + i)),
+                                    reinterpret_cast<const __half*>(blob + L.gu_biases(I + i)), H,
+                                    0, xs, lane);
     if (lane == 0) h_ws[(size_t)blockIdx.y * h_stride + i] = gelu_f(g, gelu) * u;
 }
 
@@ -87,10 +91,12 @@ k_ffn_down_simple(const MoeFfnPair* __restrict__ pairs, const float* __restrict_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = blockIdx.x * 8 + warp;
     if (r >= H) return;
-    BlobLayout L(H, I);
+    const BlobLayout L(H, I);
     const uint8_t* blob = static_cast<const uint8_t*>(pr.blob);
-    float v = q4_row_dot_warp(blob + L.dn_q, reinterpret_cast<const __half*>(blob + L.dn_s),
-                              reinterpret_cast<const __half*>(blob + L.dn_b), I, r, hs, lane);
+    const float v = q4_row_dot_warp(blob + L.dn_codes(r),
+                                    reinterpret_cast<const __half*>(blob + L.dn_scales(r)),
+                                    reinterpret_cast<const __half*>(blob + L.dn_biases(r)), I, 0,
+                                    hs, lane);
     if (lane == 0) y[(size_t)blockIdx.y * H + r] = v;
 }
 

@@ -14,15 +14,19 @@
 //   down       y = sum_e Wd_e h_e  (the routing weights are already folded
 //              into h_e, so this is the combine), h_out = fp16(h + y)
 //
-// Work items, in this order: router (8 expert rows), shared-expert gate/up
-// (16 intermediate indices = 32 rows), routed gate/up (same), down (8 output
-// rows of all k + 1 experts).  Item i belongs to CTA i mod grid, whose
-// producer warp streams its items' weights, in increasing order, into a
-// shared-memory ring with bulk asynchronous copies (TMA) and mbarriers; eight
-// consumer warps compute.  An item waits only on items of lower index
-// (routed experts on the router, down rows on every gate/up item).  Every
-// wait is bounded; on expiry the kernel records MOE_ERR_TIMEOUT in the status
-// word and drains.
+// Work items, in this order: router (2 expert rows each), shared-expert
+// gate/up (one gate/up tile: 16 intermediate indices = 32 rows), routed
+// gate/up (same), shared-expert down (32 output rows: two down tiles), routed
+// down (16 output rows of all k routed experts: one down tile of each; the
+// routing weights are folded into h, so this is the combine, and the shared
+// expert's output for the rows is added).  Item i belongs to CTA i mod grid,
+// whose producer warp streams its items' weights, in increasing order, into a
+// shared-memory ring with bulk asynchronous copies (TMA; the blob is tiled
+// so that an item is one copy, or k for a routed down item) and mbarriers;
+// eight consumer warps compute.  An item waits only on items of lower index
+// (routed items on the router, down items on their class's gate/up items,
+// routed down rows on the shared down rows).  Every wait is bounded; on
+// expiry the kernel records MOE_ERR_TIMEOUT in the status word and drains.
 //
 // Counters are monotonic (64-bit): a launch derives its epoch from one entry
 // count per CTA, so nothing has to be reset between launches.  Programmatic
@@ -36,9 +40,10 @@
 // accumulated exactly in int32 with DP4A and scaled in fp32; the fp16 group
 // bias multiplies the fp32 sum of the activations.  The input x shares one
 // exponent per 64-column group; the intermediate h shares one per 8 values,
-// packed by the warp that finishes the gate/up item.  The router dot product
-// is exact: x * 2^24 is an integer below 2^40, split into balanced base-256
-// digits.
+// packed by the warp that finishes the gate/up item, and reaches the down
+// items by one bulk copy per CTA and class once the class is published.  The
+// router dot product is exact: x * 2^24 is an integer below 2^40, split into
+// balanced base-256 digits.
 #pragma once
 #include "common.cuh"
 #include "ptx.cuh"
@@ -53,7 +58,10 @@ constexpr int kGuRows = 16;                 // intermediate indices per gate/up 
 constexpr int kRouterRows = 2;              // expert rows per router item (4 warps per row)
 constexpr int kDLimbWords = 24;             // per 32-value chunk of h: 4 x (eh oh el ol fexp sx)
 constexpr int kLimbWords = 20;              // per 32-column chunk of x in shared memory (16-byte rows)
-constexpr int kMaxDownItems = 8;            // down items one CTA keeps residual rows for
+constexpr int kMaxDownItems = 4;            // routed down items one CTA keeps residual rows for
+constexpr int kRdRows = 16;                 // output rows per routed down item (one down tile)
+constexpr int kSdRows = 32;                 // output rows per shared down item (two down tiles)
+constexpr int kRedFloats = kFusedConsumerWarps * kRdRows;   // per-stage cross-warp sums
 constexpr unsigned long long kWaitNs = 2000000000ull;   // bound of every device wait (2 s)
 
 // Work classes a launch may include (bit mask).
@@ -63,8 +71,7 @@ enum : int { kModeRouter = 1, kModeShared = 2, kModeRouted = 4, kModeDown = 8,
 struct FusedSync {               // one per launch parity; never reset
     unsigned long long entries;         // CTAs that entered: epoch = entries / grid
     unsigned long long router_done;     // router items finished
-    unsigned long long routing_ready;   // unused
-    unsigned long long gu_done;         // gate/up items finished
+    unsigned long long gu_done[2];      // gate/up items finished: [0] shared, [1] routed
     unsigned long long pad[4];
     // routing of the launch: word j < k holds expert j, word 8 + j its weight
     // bits, each tagged with (epoch + 1) in the high 32 bits, so one read of
@@ -90,17 +97,23 @@ struct FusedArgs {
     float* w_out;
     double* logits;              // [E]
     uint32_t* dlimb;             // [(k*I + Is) / 32][kDLimbWords] packed h
+    // shared-expert down output, one tagged word per row: (launch tag << 32)
+    // | fp32 bits, written by one relaxed 64-bit store
+    unsigned long long* ysh;     // [H]
+    int sync_id;                 // index of this launch's sync block (0..7), part of the tag
     FusedSync* sync;
     int* status;
     unsigned long long* trace;   // optional: kTraceWords per CTA
     double eps;
     int H, E, k, I, Is, gelu, renorm, prenorm;
     int n_stages, stage_bytes;
-    int NR, NSG, NRG, ND, NTOT;  // item counts: router, shared g/u, routed g/u, down
+    // item counts: router, shared gate/up, shared down, routed gate/up,
+    // routed down
+    int NR, NSG, NSD, NRG, NRD, NTOT;
 };
 
 struct FusedDesc {
-    int type;                    // -1 end, 0 router, 1 gate/up, 2 down
+    int type;                    // -1 end, 0 router, 1 gate/up, 2 routed down, 3 shared down
     int e_slot;                  // gate/up: 0..k-1 routed, k shared
     int blk;                     // row block
     int rows;                    // router rows in this item
@@ -451,21 +464,19 @@ __device__ __forceinline__ void fused_topk_publish(const FusedArgs& a, unsigned 
     __syncwarp();
 }
 
-// Publishes this CTA's n finished gate/up items once they are all counted in
-// *gu_done_local (bounded wait); one device-scope release.
-__device__ __forceinline__ bool fused_publish_gu(const FusedArgs& a, const volatile int* gu_done_local,
-                                                 unsigned n) {
-    if (!fused_wait_smem(gu_done_local, (int)n, a.status)) return false;
-    fence_acq_rel_gpu();
-    atomicAdd(&a.sync->gu_done, (unsigned long long)n);
-    return true;
+// Number of q in [lo, hi) with q = b (mod G).
+__device__ __forceinline__ int count_mod(int lo, int hi, int b, int G) {
+    if (hi <= lo) return 0;
+    const int first = lo + ((b - lo % G) % G + G) % G;
+    return first >= hi ? 0 : (hi - 1 - first) / G + 1;
 }
 
-// Stage layouts (bytes): router item: 8 rows of int8 [H]; gate/up item:
-// gate codes [16][H/2], up codes [16][H/2], gate scales [16][H/64] fp16, up
-// scales, gate biases, up biases (18 H in all); down item: for each expert
-// slot (routed 0..k-1, then shared, intermediate Ie) codes [8][Ie/2], scales
-// [8][Ie/64], biases [8][Ie/64] (4.5 Ie each).
+// Stage layouts (bytes): router item: kRouterRows rows of int8 [H];
+// gate/up item: one gate/up tile (gate codes [16][H/2], up codes [16][H/2],
+// gate scales [16][H/64] fp16, up scales, gate biases, up biases: 18 H);
+// shared down item: two down tiles of the shared expert (codes [16][Is/2],
+// scales [16][Is/64], biases [16][Is/64]: 9 Is each); routed down item: one
+// down tile (9 I) of each of the k routed experts, expert j at j * 9 I.
 
 // ------------------------------------------------------------- producer --
 struct ProducerShared {
@@ -520,15 +531,15 @@ __device__ __forceinline__ bool fused_get_routing(const FusedArgs& a,
 }
 
 __device__ __forceinline__ void fused_producer(const FusedArgs& a, uint8_t* stages, FusedDesc* desc,
-                                               uint64_t* full, uint64_t* empty, volatile int* gu_final,
+                                               uint64_t* full, uint64_t* empty,
                                                volatile unsigned long long* ep_slot,
                                                ProducerShared* ps, int lane) {
     const int H = a.H;
     int stage = 0;
     uint32_t phase = 0;
     uint32_t outstanding = 0, issued_parity = 0;     // bit per stage
-    bool have_routing = false, ok = true, gu_final_set = false;
-    int n_issued = 0, n_gu = 0, n_down = 0;
+    bool have_routing = false, ok = true;
+    int n_issued = 0, n_down = 0;
     for (int q = blockIdx.x; q < a.NTOT; q += gridDim.x) {
         ok = __shfl_sync(0xffffffffu, (lane == 0 && fused_aborted(a.status)) ? 0 : 1, 0) != 0;
         if (!ok) break;
@@ -539,24 +550,22 @@ __device__ __forceinline__ void fused_producer(const FusedArgs& a, uint8_t* stag
         d.item = 0;
         d.pad[0] = d.pad[1] = 0;
         bool needs_routing = false;
+        const int q1 = a.NR + a.NSG, q2 = q1 + a.NRG, q3 = q2 + a.NSD;
         if (q < a.NR) {
             d.type = 0; d.blk = q; d.rows = min(kRouterRows, a.E - kRouterRows * q);
-        } else if (q < a.NR + a.NSG) {
+        } else if (q < q1) {                                // shared gate/up tile
             d.type = 1; d.e_slot = a.k; d.blk = q - a.NR;
-        } else if (q < a.NR + a.NSG + a.NRG) {
-            const int r = q - a.NR - a.NSG;
+        } else if (q < q2) {                                // routed gate/up tile
+            const int r = q - q1;
             const int per = a.I / kGuRows;
             d.type = 1; d.e_slot = r / per; d.blk = r % per;
             needs_routing = true;
-        } else {
-            d.type = 2; d.blk = q - a.NR - a.NSG - a.NRG; d.item = n_down++;
+        } else if (q < q3) {                                // shared down: 32 rows
+            d.type = 3; d.e_slot = a.k; d.blk = q - q2;
+        } else {                                            // routed down: 16 rows x k
+            d.type = 2; d.blk = q - q3; d.item = n_down++;
             needs_routing = true;
         }
-        if (d.type != 1 && n_gu > 0 && !gu_final_set) {
-            if (lane == 0) *gu_final = n_gu;         // no gate/up item follows
-            gu_final_set = true;
-        }
-        if (d.type == 1) n_gu++;
         if (needs_routing && !have_routing) {
             if (!fused_get_routing(a, ep_slot, ps, lane)) { ok = false; break; }
             have_routing = true;
@@ -572,37 +581,27 @@ __device__ __forceinline__ void fused_producer(const FusedArgs& a, uint8_t* stag
                     const uint32_t bytes = (uint32_t)d.rows * H;
                     mbar_arrive_expect_tx(bar, bytes);
                     bulk_g2s(dst, a.Wr + (size_t)d.blk * kRouterRows * H, bytes, bar);
-                } else if (d.type == 1) {
+                } else if (d.type == 1) {                   // one gate/up tile: one copy
                     const int Ie = d.e_slot < a.k ? a.I : a.Is;
                     const uint8_t* blob = d.e_slot < a.k
                                               ? a.experts + (size_t)ps->sel[d.e_slot] * a.stride
                                               : a.shared;
                     const BlobLayout L(H, Ie);
-                    const size_t g0 = (size_t)kGuRows * d.blk, u0 = (size_t)Ie + kGuRows * d.blk;
-                    const uint32_t qb = (uint32_t)kGuRows * H / 2, sb = (uint32_t)kGuRows * H / 32;
-                    mbar_arrive_expect_tx(bar, 2 * qb + 4 * sb);
-                    bulk_g2s(dst, blob + L.gu_q + g0 * (H / 2), qb, bar);
-                    bulk_g2s(dst + qb, blob + L.gu_q + u0 * (H / 2), qb, bar);
-                    bulk_g2s(dst + 2 * qb, blob + L.gu_s + g0 * (H / 32), sb, bar);
-                    bulk_g2s(dst + 2 * qb + sb, blob + L.gu_s + u0 * (H / 32), sb, bar);
-                    bulk_g2s(dst + 2 * qb + 2 * sb, blob + L.gu_b + g0 * (H / 32), sb, bar);
-                    bulk_g2s(dst + 2 * qb + 3 * sb, blob + L.gu_b + u0 * (H / 32), sb, bar);
-                } else {
-                    const uint32_t total = (uint32_t)(9 * ((size_t)a.k * a.I + a.Is) / 2);
-                    mbar_arrive_expect_tx(bar, total);
-                    uint32_t off = 0;
-                    for (int e = 0; e <= a.k; e++) {
-                        const int Ie = e < a.k ? a.I : a.Is;
-                        const uint8_t* blob = e < a.k ? a.experts + (size_t)ps->sel[e] * a.stride
-                                                      : a.shared;
-                        const BlobLayout L(H, Ie);
-                        const size_t r0 = (size_t)8 * d.blk;
-                        const uint32_t qb = 4u * Ie, sb = (uint32_t)Ie / 4;
-                        bulk_g2s(dst + off, blob + L.dn_q + r0 * (Ie / 2), qb, bar);
-                        bulk_g2s(dst + off + qb, blob + L.dn_s + r0 * (Ie / 32), sb, bar);
-                        bulk_g2s(dst + off + qb + sb, blob + L.dn_b + r0 * (Ie / 32), sb, bar);
-                        off += qb + 2 * sb;
-                    }
+                    mbar_arrive_expect_tx(bar, (uint32_t)L.gu_tile);
+                    bulk_g2s(dst, blob + (size_t)d.blk * L.gu_tile, (uint32_t)L.gu_tile, bar);
+                } else if (d.type == 3) {                   // two shared down tiles: one copy
+                    const BlobLayout L(H, a.Is);
+                    const uint32_t bytes = 2u * (uint32_t)L.dn_tile;
+                    mbar_arrive_expect_tx(bar, bytes);
+                    bulk_g2s(dst, a.shared + L.dn_base + (size_t)(2 * d.blk) * L.dn_tile, bytes, bar);
+                } else {                                    // one down tile of each routed expert
+                    const BlobLayout L(H, a.I);
+                    mbar_arrive_expect_tx(bar, (uint32_t)(a.k * L.dn_tile));
+                    for (int e = 0; e < a.k; e++)
+                        bulk_g2s(dst + (size_t)e * L.dn_tile,
+                                 a.experts + (size_t)ps->sel[e] * a.stride + L.dn_base +
+                                     (size_t)d.blk * L.dn_tile,
+                                 (uint32_t)L.dn_tile, bar);
                 }
                 fused_trace_item(a, n_issued, 0, d.type);
             }
@@ -615,7 +614,6 @@ __device__ __forceinline__ void fused_producer(const FusedArgs& a, uint8_t* stag
         if (++stage == a.n_stages) { stage = 0; phase ^= 1u; }
     }
     if (lane != 0) return;
-    if (!gu_final_set) *gu_final = n_gu;
     fused_trace(a, kTrProducerEnd);
     // end marker for the consumers
     if (ok && fused_wait_bar(&empty[stage], phase ^ 1u, a.status)) {
@@ -639,12 +637,10 @@ struct ConsumerShared {
     double rbias[kRouterRows];
     int item_cnt[kFusedMaxStages];       // warps done with the stage's item
     int down_flag;                       // all gate/up items of the launch done
-    int gu_done_local;                   // this CTA's finished gate/up items
-    int gu_final;                        // its gate/up item count (set by the producer)
-    int gu_pub;                          // published
+    int gu_cls_done[2];                  // this CTA's finished shared / routed gate/up items
     unsigned long long ep1;              // epoch + 1 (for the producer)
     unsigned long long sc[20];           // reductions
-    __half h_rows[kMaxDownItems * 8];    // residual rows of this CTA's down items
+    __half h_rows[kMaxDownItems * kRdRows];   // residual rows of this CTA's routed down items
 };
 
 __device__ __forceinline__ FusedDesc fused_read_desc(const FusedDesc* p) {
@@ -662,7 +658,8 @@ template <int MAXC, int MAXD>
 __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* stages, FusedDesc* desc,
                                                 uint64_t* full, uint64_t* empty, __half* xs,
                                                 int8_t* xl, float* red, uint32_t* glimb,
-                                                uint8_t* hl, uint64_t* hl_bar, ConsumerShared* cs) {
+                                                uint8_t* hl, uint64_t* hl_bar, uint8_t* hls,
+                                                uint64_t* hls_bar, ConsumerShared* cs) {
     const int tid = threadIdx.x;                 // 0..255
     const int warp = tid >> 5, lane = tid & 31;
     const int H = a.H;
@@ -712,15 +709,15 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
             const int c = tid + nthr * i;
             if (c < H) xs[c] = __double2half(__dmul_rn((double)__half2float(hv[i]), r));
         }
-        // residual rows of this CTA's down items, for the final h + y
-        if (a.ND > 0) {
-            const int d0 = a.NR + a.NSG + a.NRG;
+        // residual rows of this CTA's routed down items, for the final h + y
+        if (a.NRD > 0) {
+            const int d0 = a.NR + a.NSG + a.NSD + a.NRG;
             int q0 = blockIdx.x;
             while (q0 < d0) q0 += gridDim.x;
-            for (int t = tid; t < kMaxDownItems * 8; t += nthr) {
-                const int q = q0 + (t >> 3) * gridDim.x;
+            for (int t = tid; t < kMaxDownItems * kRdRows; t += nthr) {
+                const int q = q0 + (t / kRdRows) * gridDim.x;
                 if (q < a.NTOT) {
-                    const int row = 8 * (q - d0) + (t & 7);
+                    const int row = kRdRows * (q - d0) + (t % kRdRows);
                     cs->h_rows[t] = __ushort_as_half(__ldcg((const unsigned short*)a.x_in + row));
                 }
             }
@@ -792,15 +789,23 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
     if (tid == 0) fused_trace(a, kTrProRouterLimbs);
 
 
-    // ---- h limbs for the down rows: lane owns chunk tid + 256 j of the
-    // concatenated intermediate (routed 0..k-1, then shared), loaded once
-    // every gate/up item of the launch is done
+    // ---- h limbs for the routed down rows: thread tid owns chunk tid + 256 j
+    // of the routed intermediate (experts 0..k-1), loaded once every routed
+    // gate/up item of the launch is done
     HLimbs dl[MAXD];
-    int dq_off[MAXD], ds_off[MAXD], dstride_q[MAXD], dstride_s[MAXD];
+    int dq_off[MAXD], ds_off[MAXD];
     bool dvalid[MAXD];
-    bool down_ready = false;
-    const int NC = (a.k * a.I + a.Is) / 32;
-    const unsigned long long ngu = (unsigned long long)(a.NSG + a.NRG);
+    bool down_ready = false, sdown_ready = false;
+    const int NCr = a.k * a.I / 32;                  // routed chunks
+    const int NCs = a.Is / 32;                       // shared chunks
+    // gate/up items of this CTA per class: the last of a class publishes
+    const int q1 = a.NR + a.NSG, q2 = q1 + a.NRG;
+    const int n_cls0 = count_mod(a.NR, q1, (int)blockIdx.x, (int)gridDim.x);
+    const int n_cls1 = count_mod(q1, q2, (int)blockIdx.x, (int)gridDim.x);
+    // this launch's tag of the shared down words: unique per (sync block,
+    // epoch), so a word left by an earlier launch never matches
+    const unsigned long long tag =
+        (unsigned long long)(unsigned)((ep + 1) * 8 + (unsigned long long)a.sync_id) << 32;
     unsigned cnt_r = 0, cnt_gu = 0, cnt_g = 0, cnt_d = 0;
     int n_done = 0;
     bool first = true;
@@ -815,7 +820,6 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
         if (!fused_wait_bar(&full[stage], phase, a.status)) { aborted = true; break; }
         const FusedDesc d = fused_read_desc(desc + stage);
         const uint32_t st_s = smem_u32(stages) + (uint32_t)stage * a.stage_bytes;
-        float* rs = red + (size_t)stage * 64;
         if (first) {
             if (warp == 0 && lane == 0) fused_trace(a, kTrFirstItem);
             first = false;
@@ -979,7 +983,7 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
         FusedDesc d = fused_read_desc(desc + stage);
         if (d.type < 0) break;
         const uint32_t st_s = smem_u32(stages) + (uint32_t)stage * a.stage_bytes;
-        float* rs = red + (size_t)stage * 64;
+        float* rs = red + (size_t)stage * kRedFloats;
         if (first) {
             if (warp == 0 && lane == 0) fused_trace(a, kTrFirstItem);
             first = false;
@@ -1066,31 +1070,84 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
                 if (lane == 0) {
                     cs->item_cnt[stage] = 0;
                     fence_acq_rel_cta();
-                    const int done = atomicAdd(&cs->gu_done_local, 1) + 1;
-                    const int fin = *(volatile int*)&cs->gu_final;
-                    if (fin > 0 && done == fin && atomicCAS(&cs->gu_pub, 0, 1) == 0) {
+                    // the CTA's last item of its class publishes the class
+                    const int cls = d.e_slot < a.k ? 1 : 0;
+                    const int n_c = cls ? n_cls1 : n_cls0;
+                    if (atomicAdd(&cs->gu_cls_done[cls], 1) + 1 == n_c) {
                         fence_acq_rel_gpu();
-                        atomicAdd(&a.sync->gu_done, (unsigned long long)fin);
+                        atomicAdd(&a.sync->gu_done[cls], (unsigned long long)n_c);
                     }
                 }
             }
-        } else {
-            // -------- down rows of every expert + combine
-            cnt_d++;
-            if (!down_ready) {
-                // warp 0 publishes this CTA's gate/up items if not yet done,
-                // waits for all of the launch's, then copies the packed h
-                // table into shared memory with one bulk copy; every warp
-                // waits for that copy
+        } else if (d.type == 3) {
+            // -------- shared down rows: 32 rows of the shared expert; warp w
+            // takes rows 4w..4w+3, lane l the 32-value chunks l, l + 32, ...
+            // of the shared h, whose packed limbs come into shared memory by
+            // one bulk copy once the launch's shared gate/up items are done
+            if (!sdown_ready) {
                 bool ok = true;
                 if (warp == 0 && lane == 0) {
-                    if (cnt_gu > 0 && atomicCAS(&cs->gu_pub, 0, 1) == 0)
-                        ok = fused_publish_gu(a, &cs->gu_done_local, cnt_gu);
-                    ok = ok && fused_wait_ge(&a.sync->gu_done, (ep + 1) * ngu, a.status);
+                    ok = fused_wait_ge(&a.sync->gu_done[0], (ep + 1) * (unsigned long long)a.NSG, a.status);
+                    if (ok) {
+                        fence_proxy_async_global();
+                        const uint32_t bytes = (uint32_t)NCs * kDLimbWords * 4;
+                        mbar_arrive_expect_tx(hls_bar, bytes);
+                        bulk_g2s(hls, a.dlimb + (size_t)NCr * kDLimbWords, bytes, hls_bar);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok || !fused_wait_bar(hls_bar, 0, a.status)) break;
+                sdown_ready = true;
+            }
+            const uint32_t Is = (uint32_t)a.Is, hls_s = smem_u32(hls);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int c = lane; c < NCs; c += 32) {
+                HLimbs L;
+                const uint32_t src = hls_s + (uint32_t)c * (kDLimbWords * 4);
+                const uint4 t0 = lds128(src), t1 = lds128(src + 16), t2 = lds128(src + 32),
+                            t3 = lds128(src + 48), t4 = lds128(src + 64), t5 = lds128(src + 80);
+                L.eh[0] = t0.x; L.eh[1] = t0.y; L.eh[2] = t0.z; L.eh[3] = t0.w;
+                L.oh[0] = t1.x; L.oh[1] = t1.y; L.oh[2] = t1.z; L.oh[3] = t1.w;
+                L.el[0] = t2.x; L.el[1] = t2.y; L.el[2] = t2.z; L.el[3] = t2.w;
+                L.ol[0] = t3.x; L.ol[1] = t3.y; L.ol[2] = t3.z; L.ol[3] = t3.w;
+                L.fexp[0] = __uint_as_float(t4.x); L.fexp[1] = __uint_as_float(t4.y);
+                L.fexp[2] = __uint_as_float(t4.z); L.fexp[3] = __uint_as_float(t4.w);
+                L.sx = __uint_as_float(t5.x) + __uint_as_float(t5.y) + __uint_as_float(t5.z) +
+                       __uint_as_float(t5.w);
+                const uint32_t g2 = 2u * (uint32_t)(c >> 1);
+#pragma unroll
+                for (int r = 0; r < 4; r++) {
+                    const int ir = 4 * warp + r;                      // row of the item
+                    const uint32_t tb = st_s + (uint32_t)(ir >> 4) * 9u * Is;
+                    const uint32_t j = (uint32_t)(ir & 15);
+                    const uint4 q = lds128(tb + j * (Is / 2) + 16u * (uint32_t)c);
+                    const float dd = chunk_dot_h(q, L);
+                    const uint16_t sv = lds16(tb + 8u * Is + j * (Is / 32) + g2);
+                    const uint16_t bv = lds16(tb + 8u * Is + Is / 2 + j * (Is / 32) + g2);
+                    acc[r] = fmaf(h2f_bits(sv), dd, acc[r]);
+                    acc[r] = fmaf(h2f_bits(bv), L.sx, acc[r]);
+                }
+            }
+            // lane l holds the total of row l / 8 of this warp
+            const float tot = reduce_scatter<4>(acc, lane);
+            if ((lane & 7) == 0)
+                st_relaxed_u64(a.ysh + kSdRows * d.blk + 4 * warp + (lane >> 3),
+                               tag | __float_as_uint(tot));
+        } else {
+            // -------- routed down rows + combine: 16 rows of the k routed
+            // experts (routing weights are folded into h), then + shared
+            cnt_d++;
+            if (!down_ready) {
+                // warp 0 waits for every routed gate/up item of the launch,
+                // then copies their packed h into shared memory with one bulk
+                // copy; every warp waits for that copy
+                bool ok = true;
+                if (warp == 0 && lane == 0) {
+                    ok = fused_wait_ge(&a.sync->gu_done[1], (ep + 1) * (unsigned long long)a.NRG, a.status);
                     if (ok) {
                         fused_trace(a, kTrDownReady);
                         fence_proxy_async_global();
-                        const uint32_t bytes = (uint32_t)NC * kDLimbWords * 4;
+                        const uint32_t bytes = (uint32_t)NCr * kDLimbWords * 4;
                         mbar_arrive_expect_tx(hl_bar, bytes);
                         bulk_g2s(hl, a.dlimb, bytes, hl_bar);
                     }
@@ -1098,14 +1155,13 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok || !fused_wait_bar(hl_bar, 0, a.status)) break;
                 const uint32_t hl_s = smem_u32(hl);
+                const int cpe = a.I / 32;                            // chunks per expert
 #pragma unroll
                 for (int j = 0; j < MAXD; j++) {
                     const int L = tid + 256 * j;
-                    const bool valid = L < NC;
-                    const int kI32 = a.k * (a.I / 32);
-                    const int e = !valid ? 0 : (L < kI32 ? L / (a.I / 32) : a.k);
-                    const int ce = !valid ? 0 : (e < a.k ? L - e * (a.I / 32) : L - kI32);
-                    const int Ie = e < a.k ? a.I : a.Is;
+                    const bool valid = L < NCr;
+                    const int e = valid ? L / cpe : 0;
+                    const int ce = valid ? L - e * cpe : 0;
                     uint4 t[6];
                     const uint32_t src = hl_s + (uint32_t)(valid ? L : 0) * (kDLimbWords * 4);
 #pragma unroll
@@ -1119,37 +1175,35 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
                     dl[j].sx = valid ? __uint_as_float(t[5].x) + __uint_as_float(t[5].y) +
                                        __uint_as_float(t[5].z) + __uint_as_float(t[5].w)
                                      : 0.f;
-                    const int seg = e * (9 * a.I / 2);               // shared segment follows
-                    dq_off[j] = seg + 16 * ce;
-                    ds_off[j] = seg + 4 * Ie + 2 * (ce >> 1);
-                    dstride_q[j] = Ie / 2;
-                    dstride_s[j] = Ie / 32;
+                    // expert e's down tile sits at e * 9 I in the stage
+                    dq_off[j] = e * 9 * a.I + 16 * ce;
+                    ds_off[j] = e * 9 * a.I + 8 * a.I + 2 * (ce >> 1);
                     dvalid[j] = valid;
                 }
                 down_ready = true;
                 if (tid == 0) fused_trace(a, kTrDownLimbs);
             }
-            float acc[8];
+            float acc[kRdRows];
 #pragma unroll
-            for (int r = 0; r < 8; r++) acc[r] = 0.f;
+            for (int r = 0; r < kRdRows; r++) acc[r] = 0.f;
+            const int qrow = a.I / 2, srow = a.I / 32, bo = a.I / 2;    // biases follow the scales
 #pragma unroll
             for (int j = 0; j < MAXD; j++) {
                 if (dvalid[j]) {
-                    const int bo = dstride_s[j] * 8;       // biases follow the 8 scale rows
 #pragma unroll
-                    for (int r = 0; r < 8; r++) {
-                        const uint4 q = lds128(st_s + dq_off[j] + r * dstride_q[j]);
+                    for (int r = 0; r < kRdRows; r++) {
+                        const uint4 q = lds128(st_s + dq_off[j] + r * qrow);
                         const float dd = chunk_dot_h(q, dl[j]);
-                        const uint16_t s = lds16(st_s + ds_off[j] + r * dstride_s[j]);
-                        const uint16_t b = lds16(st_s + ds_off[j] + bo + r * dstride_s[j]);
-                        acc[r] = fmaf(h2f_bits(s), dd, acc[r]);
-                        acc[r] = fmaf(h2f_bits(b), dl[j].sx, acc[r]);
+                        const uint16_t sv = lds16(st_s + ds_off[j] + r * srow);
+                        const uint16_t bv = lds16(st_s + ds_off[j] + bo + r * srow);
+                        acc[r] = fmaf(h2f_bits(sv), dd, acc[r]);
+                        acc[r] = fmaf(h2f_bits(bv), dl[j].sx, acc[r]);
                     }
                 }
             }
-            // lane l holds the total of row l / 4
-            const float tot = reduce_scatter<8>(acc, lane);
-            if ((lane & 3) == 0) rs[warp * 8 + (lane >> 2)] = tot;
+            // lane l holds the total of row l / 2
+            const float tot = reduce_scatter<kRdRows>(acc, lane);
+            if ((lane & 1) == 0) rs[warp * kRdRows + (lane >> 1)] = tot;
             __syncwarp();
             int old = 0;
             if (lane == 0) {
@@ -1159,22 +1213,41 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
             old = __shfl_sync(0xffffffffu, old, 0);
             if (old == kFusedConsumerWarps - 1) {
                 fence_acq_rel_cta();
-                if (lane < 8) {
+                bool ok = true;
+                if (lane < kRdRows) {
+                    const int row = kRdRows * d.blk + lane;
+                    // the shared expert's output for the row (written by a
+                    // shared down item of lower index; bounded wait for its tag)
+                    unsigned long long ws = ld_relaxed_u64(a.ysh + row);
+                    if ((ws & ~0xffffffffull) != tag) {
+                        const unsigned long long t0 = gtimer_ns();
+                        for (unsigned it = 0; (ws & ~0xffffffffull) != tag; it++) {
+                            __nanosleep(128);
+                            ws = ld_relaxed_u64(a.ysh + row);
+                            if ((it & 15) == 15 && (fused_aborted(a.status) || gtimer_ns() - t0 > kWaitNs)) {
+                                fused_fail(a.status);
+                                ok = false;
+                                break;
+                            }
+                        }
+                    }
                     const volatile float* vr = rs;
-                    float yv = 0.f;
+                    float yv = __uint_as_float((unsigned)ws);
 #pragma unroll
-                    for (int w = 0; w < kFusedConsumerWarps; w++) yv += vr[w * 8 + lane];
-                    const int row = 8 * d.blk + lane;
-                    a.y[row] = yv;
-                    if (a.h_out) {
-                        const __half hr = d.item < kMaxDownItems
-                                              ? cs->h_rows[8 * d.item + lane]
-                                              : __ushort_as_half(__ldcg((const unsigned short*)a.x_in + row));
-                        a.h_out[row] = __float2half_rn(__half2float(hr) + yv);
+                    for (int w = 0; w < kFusedConsumerWarps; w++) yv += vr[w * kRdRows + lane];
+                    if (ok) {
+                        a.y[row] = yv;
+                        if (a.h_out) {
+                            const __half hr = d.item < kMaxDownItems
+                                                  ? cs->h_rows[kRdRows * d.item + lane]
+                                                  : __ushort_as_half(__ldcg((const unsigned short*)a.x_in + row));
+                            a.h_out[row] = __float2half_rn(__half2float(hr) + yv);
+                        }
                     }
                 }
                 __syncwarp();
                 if (lane == 0) cs->item_cnt[stage] = 0;
+                if (!__all_sync(0xffffffffu, ok)) break;
             }
         }
         __syncwarp();
@@ -1183,9 +1256,6 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
         if (lane == 0) mbar_arrive(&empty[stage]);
         if (++stage == a.n_stages) { stage = 0; phase ^= 1u; }
     }
-    if (warp == 0 && lane == 0 && cnt_gu > 0 && !fused_aborted(a.status) &&
-        atomicCAS(&cs->gu_pub, 0, 1) == 0)
-        fused_publish_gu(a, &cs->gu_done_local, cnt_gu);
     if (warp == 0 && lane == 0 && a.trace) {
         fused_trace(a, kTrConsumerEnd);
         const unsigned cnt_s = cnt_gu - cnt_g;
@@ -1199,23 +1269,26 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
 }
 
 // Shared memory besides the stage ring: x [H] fp16, router limbs [6][H],
-// reductions [stages][64] floats, x limb table [H/32][20] words,
-// descriptors, barriers, producer and consumer scalars.
+// cross-warp sums [stages][kRedFloats], x limb table [H/32][20] words,
+// packed routed h [NCr][24] and shared h [NCs][24] words, descriptors,
+// barriers, producer and consumer scalars.
 struct FusedSmemLayout {
-    size_t xs, xl, red, glimb, hl, desc, full, empty, hlbar, ps, cs, total;
-    __host__ __device__ FusedSmemLayout(int H, int NC, int n_stages, int stage_bytes) {
+    size_t xs, xl, red, glimb, hl, hls, desc, full, empty, hlbar, hlsbar, ps, cs, total;
+    __host__ __device__ FusedSmemLayout(int H, int NCr, int NCs, int n_stages, int stage_bytes) {
         size_t off = (size_t)n_stages * stage_bytes;
-        xs = off;    off += ((size_t)H * 2 + 127) / 128 * 128;
-        xl = off;    off += ((size_t)kRouterMaxLimbs * H + 127) / 128 * 128;
-        red = off;   off += (size_t)n_stages * 64 * sizeof(float);
-        glimb = off; off += ((size_t)(H / 32) * kLimbWords * 4 + 15) / 16 * 16;
-        hl = off;    off += (size_t)NC * kDLimbWords * 4;
-        desc = off;  off += (size_t)n_stages * sizeof(FusedDesc);
-        full = off;  off += (size_t)n_stages * 8;
-        empty = off; off += (size_t)n_stages * 8;
-        hlbar = off; off += 8;
-        ps = off;    off += (sizeof(ProducerShared) + 15) / 16 * 16;
-        cs = off;    off += (sizeof(ConsumerShared) + 15) / 16 * 16;
+        xs = off;     off += ((size_t)H * 2 + 127) / 128 * 128;
+        xl = off;     off += ((size_t)kRouterMaxLimbs * H + 127) / 128 * 128;
+        red = off;    off += (size_t)n_stages * kRedFloats * sizeof(float);
+        glimb = off;  off += ((size_t)(H / 32) * kLimbWords * 4 + 15) / 16 * 16;
+        hl = off;     off += (size_t)NCr * kDLimbWords * 4;
+        hls = off;    off += (size_t)NCs * kDLimbWords * 4;
+        desc = off;   off += (size_t)n_stages * sizeof(FusedDesc);
+        full = off;   off += (size_t)n_stages * 8;
+        empty = off;  off += (size_t)n_stages * 8;
+        hlbar = off;  off += 8;
+        hlsbar = off; off += 8;
+        ps = off;     off += (sizeof(ProducerShared) + 15) / 16 * 16;
+        cs = off;     off += (sizeof(ConsumerShared) + 15) / 16 * 16;
         total = off;
     }
 };
@@ -1223,7 +1296,7 @@ struct FusedSmemLayout {
 template <int MAXC, int MAXD>
 __global__ void __launch_bounds__(kFusedThreads, 1) k_moe_layer_fused(const FusedArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const FusedSmemLayout lay(a.H, (a.k * a.I + a.Is) / 32, a.n_stages, a.stage_bytes);
+    const FusedSmemLayout lay(a.H, a.k * a.I / 32, a.Is / 32, a.n_stages, a.stage_bytes);
     uint8_t* stages = smem;
     __half* xs = reinterpret_cast<__half*>(smem + lay.xs);
     int8_t* xl = reinterpret_cast<int8_t*>(smem + lay.xl);
@@ -1234,6 +1307,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_moe_layer_fused(const Fuse
     uint64_t* empty = reinterpret_cast<uint64_t*>(smem + lay.empty);
     uint8_t* hl = smem + lay.hl;
     uint64_t* hl_bar = reinterpret_cast<uint64_t*>(smem + lay.hlbar);
+    uint8_t* hls = smem + lay.hls;
+    uint64_t* hls_bar = reinterpret_cast<uint64_t*>(smem + lay.hlsbar);
     ProducerShared* ps = reinterpret_cast<ProducerShared*>(smem + lay.ps);
     ConsumerShared* cs = reinterpret_cast<ConsumerShared*>(smem + lay.cs);
 
@@ -1246,27 +1321,27 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_moe_layer_fused(const Fuse
             for (int r = 0; r < kRouterRows; r++) cs->rsum[s][r] = 0;
         }
         mbar_init(hl_bar, 1);
+        mbar_init(hls_bar, 1);
         cs->down_flag = 0;
-        cs->gu_done_local = 0;
-        cs->gu_final = -1;
-        cs->gu_pub = 0;
+        cs->gu_cls_done[0] = cs->gu_cls_done[1] = 0;
         cs->ep1 = 0;
         fence_mbar_init();
     }
     fused_trace(a, kTrEntry);
     __syncthreads();
     if (warp == kFusedConsumerWarps) {
-        fused_producer(a, stages, desc, full, empty, &cs->gu_final,
+        fused_producer(a, stages, desc, full, empty,
                        reinterpret_cast<volatile unsigned long long*>(&cs->ep1), ps,
                        threadIdx.x & 31);
         return;
     }
-    fused_consumers<MAXC, MAXD>(a, stages, desc, full, empty, xs, xl, red, glimb, hl, hl_bar, cs);
+    fused_consumers<MAXC, MAXD>(a, stages, desc, full, empty, xs, xl, red, glimb, hl, hl_bar, hls,
+                                hls_bar, cs);
 }
 
 // Shared memory bytes besides the stage ring.
-__host__ inline size_t fused_fixed_smem(int H, int NC, int n_stages) {
-    return FusedSmemLayout(H, NC, n_stages, 0).total;
+__host__ inline size_t fused_fixed_smem(int H, int NCr, int NCs, int n_stages) {
+    return FusedSmemLayout(H, NCr, NCs, n_stages, 0).total;
 }
 
 }  // namespace moeq4

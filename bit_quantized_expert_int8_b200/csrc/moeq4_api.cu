@@ -97,6 +97,7 @@ struct moe_ctx {
     int n_sms = 0;
     bool fused_ok = false;
     uint32_t* dlimb = nullptr;         // packed intermediate of the fused kernel
+    unsigned long long* ysh = nullptr; // tagged shared-expert down output [H]
     int f_stages = 0, f_stage_bytes = 0;
     int f_regs = 0, f_max_threads = 0;
     unsigned long long* trace = nullptr;   // [n_sms * 16] phase stamps
@@ -157,15 +158,17 @@ static cudaError_t setup_fused(moe_ctx* c) {
     if (e != cudaSuccess) return e;
     const int nch = g.hidden / 32;
     const int maxc = (nch + 31) / 32;
-    const int NC = (g.top_k * g.inter + g.inter_shared) / 32;
-    const int maxd = (NC + 255) / 256;
-    size_t stage = (size_t)18 * g.hidden;                          // gate/up item
-    const size_t down = (size_t)9 * ((size_t)g.top_k * g.inter + g.inter_shared) / 2;
-    if (down > stage) stage = down;
+    const int NCr = g.top_k * g.inter / 32, NCs = g.inter_shared / 32;
+    const int maxd = (NCr + 255) / 256;
+    // a stage holds one gate/up tile (18 H bytes), two shared down tiles
+    // (18 Is) or one down tile of each routed expert (9 I k)
+    size_t stage = (size_t)18 * g.hidden;
+    if ((size_t)18 * g.inter_shared > stage) stage = (size_t)18 * g.inter_shared;
+    if ((size_t)9 * g.inter * g.top_k > stage) stage = (size_t)9 * g.inter * g.top_k;
     stage = (stage + 127) / 128 * 128;
     int ns = 0;
     for (int n = kFusedMaxStages; n >= 2 && ns == 0; n--)
-        if ((size_t)n * stage + fused_fixed_smem(g.hidden, NC, n) <= (size_t)optin) ns = n;
+        if ((size_t)n * stage + fused_fixed_smem(g.hidden, NCr, NCs, n) <= (size_t)optin) ns = n;
     c->fused_ok = g.hidden <= 4096 && maxc >= 1 && maxc <= 4 && maxd >= 1 && maxd <= 2 &&
                   ns >= 2 && stage < (1u << 20) && c->n_sms > 0;
     if (!c->fused_ok) return cudaSuccess;
@@ -187,7 +190,7 @@ static cudaError_t setup_fused(moe_ctx* c) {
     }
     c->f_stages = ns;
     c->f_stage_bytes = (int)stage;
-    c->f_smem = (size_t)ns * stage + fused_fixed_smem(g.hidden, NC, ns);
+    c->f_smem = (size_t)ns * stage + fused_fixed_smem(g.hidden, NCr, NCs, ns);
     return cudaFuncSetAttribute(c->f_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)c->f_smem);
 }
@@ -223,6 +226,7 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     size_t o_status = take(sizeof(int));
     size_t o_halt = take(H * sizeof(__half));
     size_t o_dlimb = take((k * (size_t)cfg->inter + cfg->inter_shared) / 32 * kDLimbWords * 4);
+    size_t o_ysh = take(H * sizeof(unsigned long long));
     int n_sms_dev = 0;
     cudaDeviceGetAttribute(&n_sms_dev, cudaDevAttrMultiProcessorCount, c->device);
     size_t o_trace = take((size_t)(n_sms_dev > 0 ? n_sms_dev : 1) * kTraceWords * sizeof(unsigned long long));
@@ -246,6 +250,7 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
         c->status = (int*)(c->ws + o_status);
         c->h_alt = (__half*)(c->ws + o_halt);
         c->dlimb = (uint32_t*)(c->ws + o_dlimb);
+        c->ysh = (unsigned long long*)(c->ws + o_ysh);
         c->trace = (unsigned long long*)(c->ws + o_trace);
         size_t nm = T * k * 2 + 4;
         e = cudaHostAlloc((void**)&c->miss_host, nm * sizeof(int32_t), cudaHostAllocMapped);
@@ -344,7 +349,9 @@ static int launch_fused(moe_ctx* c, const MoeLayer* L, const __half* x_in, __hal
     a.w_out = w_out;
     a.logits = c->logits;
     a.dlimb = c->dlimb;
-    a.sync = c->fsync + 2 * mi + c->fparity[mi];
+    a.ysh = c->ysh;
+    a.sync_id = 2 * mi + c->fparity[mi];
+    a.sync = c->fsync + a.sync_id;
     c->fparity[mi] ^= 1;
     a.status = c->status;
     a.trace = c->tracing ? c->trace : nullptr;
@@ -355,8 +362,9 @@ static int launch_fused(moe_ctx* c, const MoeLayer* L, const __half* x_in, __hal
     a.NR = (mode & kModeRouter) ? (g.n_experts + kRouterRows - 1) / kRouterRows : 0;
     a.NSG = (mode & kModeShared) ? g.inter_shared / kGuRows : 0;
     a.NRG = (mode & kModeRouted) ? g.top_k * (g.inter / kGuRows) : 0;
-    a.ND = (mode & kModeDown) ? g.hidden / 8 : 0;
-    a.NTOT = a.NR + a.NSG + a.NRG + a.ND;
+    a.NSD = (mode & kModeDown) ? g.hidden / kSdRows : 0;
+    a.NRD = (mode & kModeDown) ? g.hidden / kRdRows : 0;
+    a.NTOT = a.NR + a.NSG + a.NSD + a.NRG + a.NRD;
     cudaLaunchConfig_t lc{};
     lc.gridDim = dim3(c->n_sms);
     lc.blockDim = dim3(kFusedThreads);
@@ -596,6 +604,8 @@ extern "C" int moe_ctx_check(moe_ctx* c, moe_stream_t stream) {
     // context can be used again
     CK(cudaMemset(c->status, 0, sizeof(int)));
     CK(cudaMemset(c->fsync, 0, 8 * sizeof(FusedSync)));
+    // epochs restart, so tagged words of earlier launches must not survive
+    CK(cudaMemset(c->ysh, 0, (size_t)c->cfg.hidden * sizeof(unsigned long long)));
     for (int m = 0; m < 4; m++) c->fparity[m] = 0;
     return fail(st, "a bounded device wait gave up (status %d); counters reset", st);
 }

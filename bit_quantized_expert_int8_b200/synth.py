@@ -86,27 +86,34 @@ def quantize_router(w: torch.Tensor):
     return q.to(torch.int8), s16
 
 
-def blob_offsets(H: int, I: int):
-    """Byte offsets of the six sections of one expert blob and its size:
-    gate/up codes, gate/up scales, gate/up biases, down codes, down scales,
-    down biases (gate rows 0..I-1 then up rows I..2I-1)."""
-    rows = 2 * I
-    o = [0]
-    o.append(o[-1] + rows * H // 2)
-    o.append(o[-1] + rows * (H // GROUP) * 2)
-    o.append(o[-1] + rows * (H // GROUP) * 2)
-    o.append(o[-1] + H * I // 2)
-    o.append(o[-1] + H * (I // GROUP) * 2)
-    o.append(o[-1] + H * (I // GROUP) * 2)
-    return o
-
-
 def blob_bytes(H: int, I: int) -> int:
-    return blob_offsets(H, I)[-1]
+    """Size of one tiled expert blob: I/16 gate/up tiles of 18 H bytes and
+    H/16 down tiles of 9 I bytes."""
+    return (I // 16) * 18 * H + (H // 16) * 9 * I
 
 
-def _as_bytes(t: torch.Tensor) -> torch.Tensor:
-    return t.contiguous().view(torch.uint8).reshape(-1)
+def _row_bytes(t: torch.Tensor) -> torch.Tensor:
+    """[R, ...] tensor -> its bytes as uint8 [R, bytes per row]."""
+    return t.contiguous().view(torch.uint8).reshape(t.shape[0], -1)
+
+
+def pack_blob(qg, sg, bg, qd, sd, bd, H: int, I: int) -> torch.Tensor:
+    """Tiled expert blob from the quantised gate/up matrix ([2I] rows: gate
+    0..I-1, up I..2I-1) and down matrix ([H] rows).
+
+    Gate/up tile t (intermediate indices 16t..16t+15), 18 H bytes: gate
+    codes of the 16 rows, up codes of the 16 rows, gate scales, up scales,
+    gate biases, up biases.  Down tile t (output rows 16t..16t+15), 9 I
+    bytes: codes, scales, biases of the 16 rows.  Gate/up tiles first."""
+    def gu(t):
+        b = _row_bytes(t)                                   # [2I, n]
+        return b.reshape(2, I // 16, 16, -1).permute(1, 0, 2, 3).reshape(I // 16, -1)
+
+    def dn(t):
+        return _row_bytes(t).reshape(H // 16, -1)
+    tiles_gu = torch.cat([gu(qg), gu(sg), gu(bg)], dim=1)   # [I/16, 18 H]
+    tiles_dn = torch.cat([dn(qd), dn(sd), dn(bd)], dim=1)   # [H/16, 9 I]
+    return torch.cat([tiles_gu.reshape(-1), tiles_dn.reshape(-1)])
 
 
 def expert_blob(H: int, I: int, seed: int, device="cpu",
@@ -116,14 +123,11 @@ def expert_blob(H: int, I: int, seed: int, device="cpu",
     w_dn = randn((H, I), seed_for(seed, 1), device, std)
     qg, sg, bg = quantize_q4(w_gu)
     qd, sd, bd = quantize_q4(w_dn)
-    parts = [_as_bytes(t) for t in (qg, sg, bg, qd, sd, bd)]
+    blob = pack_blob(qg, sg, bg, qd, sd, bd, H, I)
+    assert blob.numel() == blob_bytes(H, I)
     if out is None:
-        return torch.cat(parts)
-    o = 0
-    for p in parts:
-        out[o:o + p.numel()].copy_(p)
-        o += p.numel()
-    assert o == out.numel()
+        return blob
+    out.copy_(blob)
     return out
 
 

@@ -127,14 +127,19 @@ const char *moe_last_error(void);
 
 /* ------------------------------------------------------------ formats --
  * Expert blob (one contiguous, 16-byte aligned buffer per expert; a blob is
- * the unit of one cache fill):
- *   [gate/up codes  u32 [2*inter][hidden/8]]  gate rows 0..inter-1,
- *                                             up rows inter..2*inter-1
- *   [gate/up scales fp16 [2*inter][hidden/64]]
- *   [gate/up biases fp16 [2*inter][hidden/64]]
- *   [down codes     u32 [hidden][inter/8]]
- *   [down scales    fp16 [hidden][inter/64]]
- *   [down biases    fp16 [hidden][inter/64]]
+ * the unit of one cache fill), stored as tiles so that each unit of work of
+ * the kernels is one contiguous read.  The gate/up matrix has 2*inter rows
+ * (gate rows 0..inter-1, up rows inter..2*inter-1) of hidden columns; the
+ * down matrix has hidden rows of inter columns.
+ *   inter/16 gate/up tiles, 18*hidden bytes each; tile t holds intermediate
+ *   indices 16t..16t+15:
+ *     [gate codes u32 [16][hidden/8]] [up codes u32 [16][hidden/8]]
+ *     [gate scales fp16 [16][hidden/64]] [up scales fp16 [16][hidden/64]]
+ *     [gate biases fp16 [16][hidden/64]] [up biases fp16 [16][hidden/64]]
+ *   then hidden/16 down tiles, 9*inter bytes each; tile t holds output rows
+ *   16t..16t+15:
+ *     [codes u32 [16][inter/8]] [scales fp16 [16][inter/64]]
+ *     [biases fp16 [16][inter/64]]
  * Weight (row r, column c) = scale[r][c/64] * code + bias[r][c/64] with
  * code = (word[r][c/8] >> 4*(c%8)) & 15: "MLX affine" 4-bit weights
  * ([RM] "L'affirmation des 2 Go ..."; [DS] "Trois optimisations cles" 1).

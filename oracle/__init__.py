@@ -54,8 +54,6 @@ def _load():
     lib.oracle_dequant.restype = dbl
     lib.oracle_blob_bytes.argtypes = [i32, i32]
     lib.oracle_blob_bytes.restype = sz
-    lib.oracle_blob_offsets.argtypes = [i32, i32, P]
-    lib.oracle_blob_offsets.restype = None
     lib.oracle_gelu.argtypes = [dbl, i32]
     lib.oracle_gelu.restype = dbl
     lib.oracle_expert_ffn.argtypes = [P, i32, i32, i32, P, P, P]
@@ -111,12 +109,6 @@ def double_to_half(v: float) -> int:
 
 def blob_bytes(H: int, I: int) -> int:
     return int(_load().oracle_blob_bytes(H, I))
-
-
-def blob_offsets(H: int, I: int) -> list[int]:
-    off = np.zeros(7, dtype=np.uint64)
-    _load().oracle_blob_offsets(H, I, _p(off))
-    return [int(v) for v in off]
 
 
 def dequant(q, scale, bias, K: int, r: int, c: int) -> float:

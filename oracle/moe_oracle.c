@@ -105,27 +105,51 @@ double oracle_dequant(const uint32_t *q, const uint16_t *scale,
 
 /* ---------------------------------------------------------- expert blob */
 
-/* Byte offsets of the six sections of one expert blob with hidden H and
- * intermediate I: gate/up codes [2I][H/8] u32 (gate rows 0..I-1, up rows
- * I..2I-1), gate/up scales [2I][H/64] fp16, gate/up biases (same), down codes
- * [H][I/8] u32, down scales [H][I/64] fp16, down biases (same). */
-void oracle_blob_offsets(int H, int I, size_t off[7])
-{
-    size_t rows_gu = 2 * (size_t)I;
-    off[0] = 0;
-    off[1] = off[0] + rows_gu * (size_t)H / 2;
-    off[2] = off[1] + rows_gu * (size_t)(H / GROUP) * 2;
-    off[3] = off[2] + rows_gu * (size_t)(H / GROUP) * 2;
-    off[4] = off[3] + (size_t)H * (size_t)I / 2;
-    off[5] = off[4] + (size_t)H * (size_t)(I / GROUP) * 2;
-    off[6] = off[5] + (size_t)H * (size_t)(I / GROUP) * 2;
-}
-
+/* Tiled expert blob with hidden H and intermediate I (the storage order is
+ * this library's own choice; the pages print none):
+ *   I/16 gate/up tiles of 18 H bytes, tile t holding intermediate indices
+ *   16t..16t+15: gate codes [16][H/8] u32, up codes [16][H/8] u32, gate
+ *   scales [16][H/64] fp16, up scales, gate biases, up biases;
+ *   then H/16 down tiles of 9 I bytes, tile t holding output rows
+ *   16t..16t+15: codes [16][I/8] u32, scales [16][I/64] fp16, biases.
+ * The gate/up matrix has 2I rows (gate rows 0..I-1, up rows I..2I-1). */
 size_t oracle_blob_bytes(int H, int I)
 {
-    size_t off[7];
-    oracle_blob_offsets(H, I, off);
-    return off[6];
+    return (size_t)(I / 16) * 18 * (size_t)H + (size_t)(H / 16) * 9 * (size_t)I;
+}
+
+/* Byte offsets of row r's codes, scales and biases: off[0..2]. */
+void oracle_gu_row(int H, int I, int r, size_t off[3])
+{
+    int up = r >= I;
+    int i = up ? r - I : r;
+    size_t tile = (size_t)(i / 16) * 18 * (size_t)H;
+    size_t row = (size_t)(16 * up + i % 16);        /* row within the tile */
+    off[0] = tile + row * (size_t)(H / 2);
+    off[1] = tile + 16 * (size_t)H + row * (size_t)(H / 32);
+    off[2] = tile + 17 * (size_t)H + row * (size_t)(H / 32);
+}
+
+void oracle_dn_row(int H, int I, int r, size_t off[3])
+{
+    size_t tile = (size_t)(I / 16) * 18 * (size_t)H + (size_t)(r / 16) * 9 * (size_t)I;
+    size_t row = (size_t)(r % 16);
+    off[0] = tile + row * (size_t)(I / 2);                 /* 16 rows of codes: 8 I bytes */
+    off[1] = tile + 8 * (size_t)I + row * (size_t)(I / 32);
+    off[2] = tile + 8 * (size_t)I + (size_t)(I / 2) + row * (size_t)(I / 32);
+}
+
+/* Weight (row r, column c) of the gate/up (dn = 0, K = H) or down (dn = 1,
+ * K = I) matrix of a blob. */
+static double blob_weight(const uint8_t *blob, int H, int I, int dn, int r, int c)
+{
+    size_t off[3];
+    if (dn)
+        oracle_dn_row(H, I, r, off);
+    else
+        oracle_gu_row(H, I, r, off);
+    return oracle_dequant((const uint32_t *)(blob + off[0]), (const uint16_t *)(blob + off[1]),
+                          (const uint16_t *)(blob + off[2]), dn ? I : H, 0, c);
 }
 
 /* ----------------------------------------------------------------- GELU */
@@ -150,22 +174,13 @@ double oracle_gelu(double g, int variant)
 void oracle_expert_ffn(const uint8_t *blob, int H, int I, int gelu,
                        const double *x, double *h_out, double *y)
 {
-    size_t off[7];
-    oracle_blob_offsets(H, I, off);
-    const uint32_t *gu_q = (const uint32_t *)(blob + off[0]);
-    const uint16_t *gu_s = (const uint16_t *)(blob + off[1]);
-    const uint16_t *gu_b = (const uint16_t *)(blob + off[2]);
-    const uint32_t *dn_q = (const uint32_t *)(blob + off[3]);
-    const uint16_t *dn_s = (const uint16_t *)(blob + off[4]);
-    const uint16_t *dn_b = (const uint16_t *)(blob + off[5]);
-
     double *h = (double *)malloc(sizeof(double) * (size_t)I);
 #pragma omp parallel for schedule(static)
     for (int i = 0; i < I; i++) {
         double g = 0.0, u = 0.0;
         for (int c = 0; c < H; c++) {
-            g += oracle_dequant(gu_q, gu_s, gu_b, H, i, c) * x[c];
-            u += oracle_dequant(gu_q, gu_s, gu_b, H, I + i, c) * x[c];
+            g += blob_weight(blob, H, I, 0, i, c) * x[c];
+            u += blob_weight(blob, H, I, 0, I + i, c) * x[c];
         }
         h[i] = oracle_gelu(g, gelu) * u;
     }
@@ -173,7 +188,7 @@ void oracle_expert_ffn(const uint8_t *blob, int H, int I, int gelu,
     for (int r = 0; r < H; r++) {
         double acc = 0.0;
         for (int i = 0; i < I; i++)
-            acc += oracle_dequant(dn_q, dn_s, dn_b, I, r, i) * h[i];
+            acc += blob_weight(blob, H, I, 1, r, i) * h[i];
         y[r] = acc;
     }
     if (h_out)

@@ -120,13 +120,31 @@ def _dense(q, s, b, rows, K):
     return sc * codes + bi
 
 
+def _tiled_rows(blob, H, I):
+    """This test's own reading of the tiled expert blob: I/16 gate/up tiles of
+    18 H bytes (gate codes, up codes, gate scales, up scales, gate biases, up
+    biases, 16 rows each), then H/16 down tiles of 9 I bytes (codes, scales,
+    biases of 16 rows).  Returns row-major byte arrays: gate/up codes,
+    scales, biases ([2I] rows, gate first), down codes, scales, biases."""
+    nt = I // 16
+    gu = blob[: nt * 18 * H].reshape(nt, 18 * H)
+
+    def rows(a, n):
+        return np.ascontiguousarray(a.reshape(nt, 2, 16, n).transpose(1, 0, 2, 3).reshape(2 * I, n))
+    q = rows(gu[:, : 16 * H], H // 2)
+    sc = rows(gu[:, 16 * H: 17 * H], H // 32)
+    bi = rows(gu[:, 17 * H:], H // 32)
+    dn = blob[nt * 18 * H:].reshape(H // 16, 9 * I)
+    dq = np.ascontiguousarray(dn[:, : 8 * I]).reshape(H, I // 2)
+    ds = np.ascontiguousarray(dn[:, 8 * I: 8 * I + I // 2]).reshape(H, I // 32)
+    db = np.ascontiguousarray(dn[:, 8 * I + I // 2:]).reshape(H, I // 32)
+    return q, sc, bi, dq, ds, db
+
+
 def _blob_parts(blob, H, I):
-    o = synth.blob_offsets(H, I)
-    sec = [blob[o[i]:o[i + 1]] for i in range(6)]
-    Wgu = _dense(sec[0].view(np.uint32), sec[1].view(np.uint16),
-                 sec[2].view(np.uint16), 2 * I, H)
-    Wd = _dense(sec[3].view(np.uint32), sec[4].view(np.uint16),
-                sec[5].view(np.uint16), H, I)
+    q, sc, bi, dq, ds, db = _tiled_rows(blob, H, I)
+    Wgu = _dense(q.view(np.uint32), sc.view(np.uint16), bi.view(np.uint16), 2 * I, H)
+    Wd = _dense(dq.view(np.uint32), ds.view(np.uint16), db.view(np.uint16), H, I)
     return Wgu[:I], Wgu[I:], Wd
 
 
@@ -151,19 +169,20 @@ def test_expert_ffn_against_dense_brute_force(H, I, variant):
 
 def test_expert_ffn_closed_forms():
     H, I = 64, 64
-    o = synth.blob_offsets(H, I)
-    blob = np.zeros(o[-1], np.uint8)
+    blob = np.zeros(synth.blob_bytes(H, I), np.uint8)
     x = np.random.default_rng(3).standard_normal(H)
     # all-zero weights (scale 0, bias 0) -> h = 0, y = 0
     y, h = oracle.expert_ffn(blob, H, I, x)
     assert not y.any() and not h.any()
     # every weight equal: gate = up = w0 * sum(x); down weights all w1
     w0, w1 = 0.25, -0.5
-    blob[o[0]:o[1]] = 0x33                    # every code 3
-    blob[o[1]:o[2]] = np.tile(h16([0.0625]).view(np.uint8), (o[2] - o[1]) // 2)
-    blob[o[2]:o[3]] = np.tile(h16([0.0625]).view(np.uint8), (o[3] - o[2]) // 2)
+    nt = I // 16
+    gu = blob[: nt * 18 * H].reshape(nt, 18 * H)
+    gu[:, : 16 * H] = 0x33                    # every code 3
+    gu[:, 16 * H:] = np.tile(h16([0.0625]).view(np.uint8), H)   # scales and biases 1/16
     # down: code 0 everywhere, bias w1
-    blob[o[5]:o[6]] = np.tile(h16([w1]).view(np.uint8), (o[6] - o[5]) // 2)
+    dn = blob[nt * 18 * H:].reshape(H // 16, 9 * I)
+    dn[:, 8 * I + I // 2:] = np.tile(h16([w1]).view(np.uint8), I // 4)
     y, h = oracle.expert_ffn(blob, H, I, x)
     g = w0 * x.sum()
     assert np.allclose(h, oracle.gelu(g, 0) * g, rtol=1e-13)
