@@ -55,6 +55,24 @@ def env_rank():
             int(os.environ.get("WORLD_SIZE", 1)))
 
 
+def max_over_ranks(value, world, device):
+    """The largest value over all ranks (a time: the job ends with its slowest
+    rank).  With one rank, the value itself."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, tokens_per_rank, ms_max):
+    """Whole-job throughput: every rank decodes its own tokens (replicas), the
+    job takes as long as its slowest rank."""
+    return world * tokens_per_rank / (ms_max / 1000.0)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -175,18 +193,17 @@ def run_ours(args):
     clocks = ClockSampler(local_rank)
     clocks.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.profiler.start()          # a profiler started with capture off records this region
     e0.record(stream)
     for _ in range(args.steps):
         step()
     e1.record(stream)
     barrier()
+    torch.cuda.profiler.stop()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1) / args.steps
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
-    value = world * T / (ms_max / 1000.0)
+    ms_max = max_over_ranks(ms, world, dev)
+    value = job_tokens_per_s(world, T, ms_max)
 
     # ---- end to end through the C ABI with host buffers
     h_host = h0.cpu().pin_memory()
@@ -206,10 +223,7 @@ def run_ours(args):
     e1.record(stream)
     barrier()
     ms_e2e = e0.elapsed_time(e1) / args.steps
-    t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_value = world * T / (float(t.item()) / 1000.0)
+    e2e_value = job_tokens_per_s(world, T, max_over_ranks(ms_e2e, world, dev))
 
     moeq4.moe_ctx_check(ctx)
     # ---- dominant kernel: the fused layer kernel of one token-layer
@@ -246,6 +260,24 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+# DRAM bytes (read + write) of one launch of the fused layer kernel, from an
+# ncu capture of the kernel built from the source with this SHA-256; any other
+# source reports null (the counters describe a different kernel).
+KERNEL_SRC = os.path.join(ROOT, "bit_quantized_expert_int8_b200", "csrc", "layer_fused.cuh")
+TRAFFIC_BY_SOURCE = {
+    # ncu --set full, one launch of the 30-layer bench layers (hidden 2816,
+    # top-8): dram__bytes_read.sum 37,284,864 + dram__bytes_write.sum 43,008
+    "ab523b1bf6c48f302f20a8d0fa33bdea867f6816a4e0a6fbc4a69b12422ad079": 37327872,
+}
+
+
+def kernel_traffic():
+    import hashlib
+    with open(KERNEL_SRC, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    return TRAFFIC_BY_SOURCE.get(digest), digest
 
 
 def roofline(ctx, layers, cfg, dev, stream):
@@ -289,7 +321,7 @@ def roofline(ctx, layers, cfg, dev, stream):
             "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(achieved / hbm, 4), "peak_kind": f"{kind} (hbm_gbs)",
             "algorithmic_bytes_per_launch": algo, "us_per_launch": round(us, 3),
-            "traffic": None}
+            "traffic": kernel_traffic()[0]}
 
 
 def cpu_baseline(layers, cfg, seconds, h0=None, n_sample_layers=2):
