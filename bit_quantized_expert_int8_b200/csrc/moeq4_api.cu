@@ -12,6 +12,7 @@
 
 #include "common.cuh"
 #include "ffn_simple.cuh"
+#include "grouped.cuh"
 #include "layer_fused.cuh"
 #include "misc.cuh"
 #include "router.cuh"
@@ -96,6 +97,9 @@ struct moe_ctx {
     int fparity[4] = {0, 0, 0, 0};
     int n_sms = 0;
     bool fused_ok = false;
+    bool grouped_ok = false;           // multi-token steps grouped by expert
+    int* e_off = nullptr;              // [E + 1] pairs per expert (prefix)
+    int* plist = nullptr;              // [maxT * k] pair indices grouped by expert
     uint32_t* dlimb = nullptr;         // packed intermediate of the fused kernel
     unsigned long long* ysh = nullptr; // tagged shared-expert down output [H]
     int f_stages = 0, f_stage_bytes = 0;
@@ -147,6 +151,31 @@ extern "C" int moe_ctx_destroy(moe_ctx* c) {
     if (c->ws) cudaFree(c->ws);
     delete c;
     return MOE_OK;
+}
+
+// Shared memory of the grouped kernels: the expert tile plus kGrpTokens rows
+// of activations (fp32).
+static size_t grouped_smem_gu(int H) { return (size_t)18 * H + (size_t)kGrpTokens * H * 4; }
+static size_t grouped_smem_dn(int Ie) { return (size_t)9 * Ie + (size_t)kGrpTokens * Ie * 4; }
+
+// Enables the grouped multi-token path when its tiles fit shared memory.
+static cudaError_t setup_grouped(moe_ctx* c) {
+    const MoeConfig& g = c->cfg;
+    int optin = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, c->device);
+    if (e != cudaSuccess) return e;
+    const size_t gu = grouped_smem_gu(g.hidden);
+    const size_t dn = grouped_smem_dn(c->maxI);
+    c->grouped_ok = gu <= (size_t)optin && dn <= (size_t)optin;
+    if (!c->grouped_ok) return cudaSuccess;
+    e = cudaFuncSetAttribute(k_gateup_grouped<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gu);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_gateup_grouped<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gu);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_down_grouped<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_down_grouped<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn);
+    return e;
 }
 
 // Chooses the fused kernel variant and its shared-memory ring for cfg.
@@ -227,6 +256,8 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     size_t o_halt = take(H * sizeof(__half));
     size_t o_dlimb = take((k * (size_t)cfg->inter + cfg->inter_shared) / 32 * kDLimbWords * 4);
     size_t o_ysh = take(H * sizeof(unsigned long long));
+    size_t o_eoff = take((E + 1) * sizeof(int));
+    size_t o_plist = take(T * k * sizeof(int));
     int n_sms_dev = 0;
     cudaDeviceGetAttribute(&n_sms_dev, cudaDevAttrMultiProcessorCount, c->device);
     size_t o_trace = take((size_t)(n_sms_dev > 0 ? n_sms_dev : 1) * kTraceWords * sizeof(unsigned long long));
@@ -239,6 +270,8 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
         c->idx = (int32_t*)(c->ws + o_idx);
         c->w = (float*)(c->ws + o_w);
         c->pairs = (MoeFfnPair*)(c->ws + o_pairs);
+        c->e_off = (int*)(c->ws + o_eoff);
+        c->plist = (int*)(c->ws + o_plist);
         c->h_ws = (float*)(c->ws + o_h);
         c->y_pairs = (float*)(c->ws + o_y);
         c->x_norm = (__half*)(c->ws + o_xn);
@@ -272,6 +305,7 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_ffn_down_simple, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)(c->maxI * sizeof(float)));
+    if (e == cudaSuccess) e = setup_grouped(c);
     if (e == cudaSuccess) e = setup_fused(c);
     if (e != cudaSuccess) {
         rc = fail(MOE_ERR_CUDA, "moe_ctx_create: %s", cudaGetErrorString(e));
@@ -471,11 +505,33 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
     TRY(launch_router(c, L->router_w, L->router_scale, L->router_bias, xin, T, idx, w, nullptr, s));
     const size_t stride = BlobLayout(H, g.inter).bytes;
     const int P = T * (k + 1);
-    k_build_pairs<<<(P + 127) / 128, 128, 0, s>>>(L->shared_blob, g.inter_shared,
-                                                  static_cast<const uint8_t*>(L->experts), stride,
-                                                  idx, g.inter, T, k, c->pairs);
-    CKL();
-    TRY(launch_ffn(c, c->pairs, P, xin, T, c->h_ws, c->y_pairs, s));
+    if (c->grouped_ok) {
+        // each expert read once for all of its tokens
+        const uint8_t* ex = static_cast<const uint8_t*>(L->experts);
+        const uint8_t* sh = static_cast<const uint8_t*>(L->shared_blob);
+        const int E = g.n_experts, I = g.inter, Is = g.inter_shared;
+        k_group_pairs<<<1, 1024, 0, s>>>(idx, T * k, E, c->e_off, c->plist);
+        CKL();
+        k_gateup_grouped<false><<<dim3(I / 16, E), kGrpThreads, grouped_smem_gu(H), s>>>(
+            ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, g.gelu, c->h_ws, c->maxI);
+        CKL();
+        const int chunks = (T + kGrpChunk - 1) / kGrpChunk;
+        k_gateup_grouped<true><<<dim3(Is / 16, 1, chunks), kGrpThreads, grouped_smem_gu(H), s>>>(
+            ex, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, g.gelu, c->h_ws, c->maxI);
+        CKL();
+        k_down_grouped<false><<<dim3(H / 16, E), kGrpThreads, grouped_smem_dn(I), s>>>(
+            ex, stride, sh, H, I, T, c->e_off, c->plist, c->h_ws, c->maxI, c->y_pairs);
+        CKL();
+        k_down_grouped<true><<<dim3(H / 16, 1, chunks), kGrpThreads, grouped_smem_dn(Is), s>>>(
+            ex, stride, sh, H, Is, T, c->e_off, c->plist, c->h_ws, c->maxI, c->y_pairs);
+        CKL();
+    } else {
+        k_build_pairs<<<(P + 127) / 128, 128, 0, s>>>(L->shared_blob, g.inter_shared,
+                                                      static_cast<const uint8_t*>(L->experts), stride,
+                                                      idx, g.inter, T, k, c->pairs);
+        CKL();
+        TRY(launch_ffn(c, c->pairs, P, xin, T, c->h_ws, c->y_pairs, s));
+    }
     TRY(launch_combine(c, c->y_pairs + (size_t)T * H, c->y_pairs, w, T, o->y,
                        (flags & MOE_PRENORM) ? x : nullptr, s));
     return MOE_OK;

@@ -205,6 +205,34 @@ def test_layer_resident_parity(cfg, T, bias):
         assert_y_close(y[t].cpu().numpy(), ref["y"], f"token {t}")
 
 
+@pytest.mark.parametrize("cfg,T,bias,sample", [(LAYER, 40, 1.5, (0, 13, 27, 39)),
+                                               (LAYER, 2, None, (0, 1)),
+                                               (SMALL, 33, 0.7, tuple(range(33)))])
+def test_layer_grouped_multi_token(cfg, T, bias, sample):
+    """T > 1 runs the grouped path (each expert read once for all of its
+    tokens, tokens in passes of 4, ragged last pass); sampled tokens against
+    the oracle, and the same step split into single-token calls."""
+    L = make_layer(cfg, seed=4, bias_std=bias)
+    x = synth.tokens(T, cfg.H, seed=14, device=DEV)
+    ctx = ctx_for(cfg, T)
+    lay = moeq4.Layer.from_dict(L)
+    y = torch.empty((T, cfg.H), device=DEV)
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device=DEV)
+    moeq4.moe_layer_decode(ctx, lay, x, T, y, idx)
+    torch.cuda.synchronize()
+    Ln = np_layer(L)
+    xn = np_of(x)
+    for t in sample:
+        ref = _oracle_layer(cfg, Ln, xn[t])
+        assert idx[t].cpu().tolist() == ref["idx"].tolist()
+        assert_y_close(y[t].cpu().numpy(), ref["y"], f"token {t}")
+    y1 = torch.empty((1, cfg.H), device=DEV)
+    for t in sample[:2]:
+        moeq4.moe_layer_decode(ctx, lay, x[t:t + 1], 1, y1)
+        torch.cuda.synchronize()
+        assert_y_close(y1[0].cpu().numpy(), y[t].cpu().numpy().astype(np.float64), f"single {t}")
+
+
 def test_layer_prenorm_rmsnorm_exact_and_residual():
     cfg = SMALL
     T = 4
