@@ -526,7 +526,7 @@ def run_batched(args):
                       "distinct_experts": round(touched, 1), "algorithmic_bytes": int(algo),
                       "achieved_gbs": round(algo / (us * 1e-6) / 1e9, 1),
                       "frac_of_hbm": round(algo / (us * 1e-6) / 1e9 / hbm, 4),
-                      "path": "fused single-token kernel" if T == 1 else "direct kernels"})
+                      "path": "fused single-token kernel" if T == 1 else "grouped kernels"})
     moeq4.moe_ctx_check(ctx)
     print(json.dumps({"metric": METRIC, "workload": "batched sweep, one layer", "unit": UNIT,
                       "peak_gbs": hbm, "peak_kind": kind, "sweep": lines}), flush=True)
