@@ -186,11 +186,13 @@ __device__ __forceinline__ void grp_stage_float(float* xsf, int K, const float* 
 // step's tokens).  grid (Ie / 16, n_experts or 1, 1 or chunks), block 256; dynamic shared
 // memory 18 H + kGrpTokens * H * 4 bytes.  Warp w: indices 2w, 2w + 1 (gate
 // rows w-pair, up rows w-pair); lane l: 8-column words l, l + 32, ...
+// A routed expert whose bucket holds n_cap or more pairs is skipped (the
+// tensor-core kernel takes it).
 template <bool SHARED>
 __global__ void __launch_bounds__(kGrpThreads, 2)
 k_gateup_grouped(const uint8_t* __restrict__ experts, size_t stride, const uint8_t* __restrict__ shared_blob,
                  int H, int Ie, const __half* __restrict__ x, int T, int k,
-                 const int* __restrict__ e_off, const int* __restrict__ list, int gelu,
+                 const int* __restrict__ e_off, const int* __restrict__ list, int n_cap, int gelu,
                  float* __restrict__ h_ws, int h_stride) {
     extern __shared__ __align__(16) uint8_t gsm[];
     int n = T, base = 0, z0 = 0;
@@ -198,7 +200,7 @@ k_gateup_grouped(const uint8_t* __restrict__ experts, size_t stride, const uint8
     if (!SHARED) {
         base = e_off[blockIdx.y];
         n = e_off[blockIdx.y + 1] - base;
-        if (n == 0) return;
+        if (n == 0 || n >= n_cap) return;                 // empty, or left to the tensor cores
         blob = experts + (size_t)blockIdx.y * stride;
     } else {
         z0 = blockIdx.z * kGrpChunk;                      // this CTA's tokens
@@ -254,19 +256,20 @@ k_gateup_grouped(const uint8_t* __restrict__ experts, size_t stride, const uint8
 // tokens (the shared expert: kGrpChunk tokens per CTA, grid z).  grid
 // (H / 16, n_experts or 1, 1 or chunks), block 256; dynamic shared memory
 // 9 Ie + kGrpTokens * Ie * 4 bytes.  Warp w: tile rows 2w, 2w + 1; lane l:
-// 8-column words l, l + 32, ... of the intermediate.
+// 8-column words l, l + 32, ... of the intermediate.  Routed buckets of n_cap or more
+// pairs are skipped, as in the gate/up kernel.
 template <bool SHARED>
 __global__ void __launch_bounds__(kGrpThreads, 2)
 k_down_grouped(const uint8_t* __restrict__ experts, size_t stride, const uint8_t* __restrict__ shared_blob,
                int H, int Ie, int T, const int* __restrict__ e_off, const int* __restrict__ list,
-               const float* __restrict__ h_ws, int h_stride, float* __restrict__ y_pairs) {
+               int n_cap, const float* __restrict__ h_ws, int h_stride, float* __restrict__ y_pairs) {
     extern __shared__ __align__(16) uint8_t gsm[];
     int n = T, base = 0, z0 = 0;
     const uint8_t* blob = shared_blob;
     if (!SHARED) {
         base = e_off[blockIdx.y];
         n = e_off[blockIdx.y + 1] - base;
-        if (n == 0) return;
+        if (n == 0 || n >= n_cap) return;                 // empty, or left to the tensor cores
         blob = experts + (size_t)blockIdx.y * stride;
     } else {
         z0 = blockIdx.z * kGrpChunk;                      // this CTA's tokens

@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "ffn_mma.cuh"
 #include "ffn_simple.cuh"
 #include "grouped.cuh"
 #include "layer_fused.cuh"
@@ -98,6 +99,8 @@ struct moe_ctx {
     int n_sms = 0;
     bool fused_ok = false;
     bool grouped_ok = false;           // multi-token steps grouped by expert
+    bool mma_ok = false;               // tensor-core kernels usable for this shape
+    int mma_min_tok = 0;               // bucket size from which they run (0: never)
     int* e_off = nullptr;              // [E + 1] pairs per expert (prefix)
     int* plist = nullptr;              // [maxT * k] pair indices grouped by expert
     uint32_t* dlimb = nullptr;         // packed intermediate of the fused kernel
@@ -175,7 +178,20 @@ static cudaError_t setup_grouped(moe_ctx* c) {
         e = cudaFuncSetAttribute(k_down_grouped<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_down_grouped<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn);
-    return e;
+    if (e != cudaSuccess) return e;
+    // tensor-core kernels: 4 gate/up tiles (64 indices) or 128 down rows per CTA
+    if (kMmaSmem > optin || g.hidden % kMmaRows || g.inter % 64 || g.inter_shared % 64) return cudaSuccess;
+    e = cudaFuncSetAttribute(k_ffn_mma<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMmaSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_ffn_mma<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMmaSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_ffn_mma<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMmaSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_ffn_mma<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMmaSmem);
+    if (e != cudaSuccess) return e;
+    c->mma_ok = true;
+    c->mma_min_tok = kMmaDefaultMinTokens;
+    return cudaSuccess;
 }
 
 // Chooses the fused kernel variant and its shared-memory ring for cfg.
@@ -510,20 +526,49 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
         const uint8_t* ex = static_cast<const uint8_t*>(L->experts);
         const uint8_t* sh = static_cast<const uint8_t*>(L->shared_blob);
         const int E = g.n_experts, I = g.inter, Is = g.inter_shared;
+        // buckets of tau or more pairs go to the tensor cores (tau = 0: none)
+        const int tau = c->mma_ok ? c->mma_min_tok : 0;
+        const bool mma_routed = tau > 0 && T >= tau, mma_shared = tau > 0 && T >= tau;
+        const int cap = mma_routed ? tau : 0x7fffffff;
+        const int tiles = (T + kMmaTok - 1) / kMmaTok;
         k_group_pairs<<<1, 1024, 0, s>>>(idx, T * k, E, c->e_off, c->plist);
         CKL();
         k_gateup_grouped<false><<<dim3(I / 16, E), kGrpThreads, grouped_smem_gu(H), s>>>(
-            ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, g.gelu, c->h_ws, c->maxI);
+            ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
         CKL();
+        if (mma_routed) {
+            k_ffn_mma<false, false><<<dim3(I / 64, E, tiles), kMmaThreads, kMmaSmem, s>>>(
+                ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, tau, g.gelu, c->h_ws, c->maxI,
+                c->y_pairs, c->status);
+            CKL();
+        }
         const int chunks = (T + kGrpChunk - 1) / kGrpChunk;
-        k_gateup_grouped<true><<<dim3(Is / 16, 1, chunks), kGrpThreads, grouped_smem_gu(H), s>>>(
-            ex, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, g.gelu, c->h_ws, c->maxI);
+        if (mma_shared) {
+            k_ffn_mma<false, true><<<dim3(Is / 64, 1, tiles), kMmaThreads, kMmaSmem, s>>>(
+                ex, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, tau, g.gelu, c->h_ws, c->maxI,
+                c->y_pairs, c->status);
+        } else {
+            k_gateup_grouped<true><<<dim3(Is / 16, 1, chunks), kGrpThreads, grouped_smem_gu(H), s>>>(
+                ex, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
+        }
         CKL();
         k_down_grouped<false><<<dim3(H / 16, E), kGrpThreads, grouped_smem_dn(I), s>>>(
-            ex, stride, sh, H, I, T, c->e_off, c->plist, c->h_ws, c->maxI, c->y_pairs);
+            ex, stride, sh, H, I, T, c->e_off, c->plist, cap, c->h_ws, c->maxI, c->y_pairs);
         CKL();
-        k_down_grouped<true><<<dim3(H / 16, 1, chunks), kGrpThreads, grouped_smem_dn(Is), s>>>(
-            ex, stride, sh, H, Is, T, c->e_off, c->plist, c->h_ws, c->maxI, c->y_pairs);
+        if (mma_routed) {
+            k_ffn_mma<true, false><<<dim3(H / kMmaRows, E, tiles), kMmaThreads, kMmaSmem, s>>>(
+                ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, tau, g.gelu, c->h_ws, c->maxI,
+                c->y_pairs, c->status);
+            CKL();
+        }
+        if (mma_shared) {
+            k_ffn_mma<true, true><<<dim3(H / kMmaRows, 1, tiles), kMmaThreads, kMmaSmem, s>>>(
+                ex, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, tau, g.gelu, c->h_ws, c->maxI,
+                c->y_pairs, c->status);
+        } else {
+            k_down_grouped<true><<<dim3(H / 16, 1, chunks), kGrpThreads, grouped_smem_dn(Is), s>>>(
+                ex, stride, sh, H, Is, T, c->e_off, c->plist, cap, c->h_ws, c->maxI, c->y_pairs);
+        }
         CKL();
     } else {
         k_build_pairs<<<(P + 127) / 128, 128, 0, s>>>(L->shared_blob, g.inter_shared,
@@ -648,6 +693,15 @@ extern "C" int moe_layer_decode(moe_ctx* c, const MoeLayer* L, moe_half* x, int 
     if (!aligned16(L->slots) || !aligned16(L->lfu) || !aligned16(L->host_store))
         return fail(MOE_ERR_ALIGNMENT, "moe_layer_decode: pointers must be 16-byte aligned");
     return layer_streaming(c, L, reinterpret_cast<__half*>(x), o, flags, main, copy);
+}
+
+extern "C" int moe_set_mma_min_tokens(moe_ctx* c, int min_tokens) {
+    if (!c) return fail(MOE_ERR_INVALID_ARG, "moe_set_mma_min_tokens: NULL context");
+    if (min_tokens < 0) return fail(MOE_ERR_INVALID_ARG, "moe_set_mma_min_tokens: %d < 0", min_tokens);
+    if (min_tokens > 0 && !c->mma_ok)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "tensor-core kernels unavailable for this shape");
+    c->mma_min_tok = min_tokens;
+    return MOE_OK;
 }
 
 extern "C" int moe_ctx_check(moe_ctx* c, moe_stream_t stream) {

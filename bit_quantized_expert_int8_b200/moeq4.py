@@ -31,7 +31,7 @@ EXPORTS = ("moe_ctx_create", "moe_ctx_destroy", "moe_ctx_check", "moe_ctx_trace"
            "moe_last_error", "moe_blob_bytes",
            "moe_router_topk", "moe_expert_ffn_q4", "moe_combine", "moe_lfu_init",
            "moe_cache_lookup_lfu", "moe_layer_decode", "moe_stack_decode",
-           "moe_router_topk_noalloc")
+           "moe_router_topk_noalloc", "moe_set_mma_min_tokens")
 
 
 class MoeError(RuntimeError):
@@ -90,6 +90,7 @@ def load() -> ctypes.CDLL:
         "moe_ctx_check": ([P, P], i32),
         "moe_ctx_trace": ([P, i32, P, i32], i32),
         "moe_ctx_info": ([P, ctypes.c_char_p, i32], i32),
+        "moe_set_mma_min_tokens": ([P, i32], i32),
         "moe_last_error": ([], ctypes.c_char_p),
         "moe_blob_bytes": ([i32, i32], ctypes.c_size_t),
         "moe_router_topk": ([P, P, P, P, P, i32, P, P, P, P], i32),
@@ -176,6 +177,12 @@ def moe_ctx_info(ctx) -> str:
     buf = ctypes.create_string_buffer(512)
     _check(load().moe_ctx_info(ctx.handle, buf, 512))
     return buf.value.decode()
+
+
+def moe_set_mma_min_tokens(ctx, min_tokens: int):
+    """moe_set_mma_min_tokens: bucket size from which multi-token steps run
+    an expert on the tensor cores (0: never)."""
+    _check(load().moe_set_mma_min_tokens(ctx.handle, int(min_tokens)))
 
 
 def moe_ctx_trace(ctx, enable=-1, read=False):

@@ -109,6 +109,20 @@ int moe_ctx_check(moe_ctx *ctx, moe_stream_t stream);
  * len bytes (NUL-terminated) into buf (host). */
 int moe_ctx_info(moe_ctx *ctx, char *buf, int len);
 
+/* Multi-token steps with all experts resident group the (token, expert)
+ * pairs by expert ("Gemma 4 26B : Comment faire tourner un LLM en 2 Go de
+ * RAM", section 04 "Chunked Prefill": one expert applied to many rows).  An
+ * expert whose bucket holds min_tokens or more pairs (and the shared expert,
+ * once T >= min_tokens) runs on the tensor cores (tcgen05, bf16 hi/lo split
+ * of weights and activations, fp32 accumulation); smaller buckets run on the
+ * CUDA-core grouped kernels.  min_tokens = 0 keeps every bucket on the CUDA
+ * cores.  The default is 32 where the shape allows the tensor-core kernels
+ * (hidden a multiple of 128), else 0.  Host call, no device work.  Returns
+ * MOE_ERR_INVALID_ARG for min_tokens < 0 and MOE_ERR_UNSUPPORTED_SHAPE for
+ * min_tokens > 0 on a shape or device without the tensor-core kernels (the
+ * setting is then left unchanged). */
+int moe_set_mma_min_tokens(moe_ctx *ctx, int min_tokens);
+
 /* Tracing of the single-token layer kernel.  enable = 1 makes later launches
  * record, per CTA, 160 words: globaltimer stamps (ns) of kernel entry, end of
  * the input prologue, first item, routing known, down phase ready, consumer
