@@ -101,6 +101,10 @@ struct moe_ctx {
     bool grouped_ok = false;           // multi-token steps grouped by expert
     bool mma_ok = false;               // tensor-core kernels usable for this shape
     int mma_min_tok = 0;               // bucket size from which they run (0: never)
+    __nv_bfloat16* x_pl = nullptr;     // [2][maxT][H] x as bf16 hi / lo planes
+    __nv_bfloat16* h_pl = nullptr;     // [2][maxT * (k + 1)][maxI] h as bf16 hi / lo planes
+    float* x_sum = nullptr;            // [maxT][H / 64] 64-column group sums of x
+    float* h_sum = nullptr;            // [maxT * (k + 1)][maxI / 64] group sums of h
     int* e_off = nullptr;              // [E + 1] pairs per expert (prefix)
     int* plist = nullptr;              // [maxT * k] pair indices grouped by expert
     uint32_t* dlimb = nullptr;         // packed intermediate of the fused kernel
@@ -180,14 +184,17 @@ static cudaError_t setup_grouped(moe_ctx* c) {
         e = cudaFuncSetAttribute(k_down_grouped<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn);
     if (e != cudaSuccess) return e;
     // tensor-core kernels: 4 gate/up tiles (64 indices) or 128 down rows per CTA
-    if (kMmaSmem > optin || g.hidden % kMmaRows || g.inter % 64 || g.inter_shared % 64) return cudaSuccess;
-    e = cudaFuncSetAttribute(k_ffn_mma<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMmaSmem);
+    const size_t sm_gu = mma_smem_bytes(g.hidden), sm_dn = mma_smem_bytes(c->maxI);
+    if (sm_gu > (size_t)optin || sm_dn > (size_t)optin || g.hidden % kMmaRows || g.inter % 64 ||
+        g.inter_shared % 64)
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(k_ffn_mma<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_gu);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_ffn_mma<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMmaSmem);
+        e = cudaFuncSetAttribute(k_ffn_mma<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_gu);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_ffn_mma<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMmaSmem);
+        e = cudaFuncSetAttribute(k_ffn_mma<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dn);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_ffn_mma<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMmaSmem);
+        e = cudaFuncSetAttribute(k_ffn_mma<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dn);
     if (e != cudaSuccess) return e;
     c->mma_ok = true;
     c->mma_min_tok = kMmaDefaultMinTokens;
@@ -274,6 +281,10 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     size_t o_ysh = take(H * sizeof(unsigned long long));
     size_t o_eoff = take((E + 1) * sizeof(int));
     size_t o_plist = take(T * k * sizeof(int));
+    size_t o_xpl = take(2 * T * H * sizeof(__nv_bfloat16));                 // x hi / lo planes
+    size_t o_hpl = take(2 * P * (size_t)c->maxI * sizeof(__nv_bfloat16));   // h hi / lo planes
+    size_t o_xsum = take(T * (H / 64) * sizeof(float));                      // x group sums
+    size_t o_hsum = take(P * (size_t)(c->maxI / 64) * sizeof(float));        // h group sums
     int n_sms_dev = 0;
     cudaDeviceGetAttribute(&n_sms_dev, cudaDevAttrMultiProcessorCount, c->device);
     size_t o_trace = take((size_t)(n_sms_dev > 0 ? n_sms_dev : 1) * kTraceWords * sizeof(unsigned long long));
@@ -288,6 +299,10 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
         c->pairs = (MoeFfnPair*)(c->ws + o_pairs);
         c->e_off = (int*)(c->ws + o_eoff);
         c->plist = (int*)(c->ws + o_plist);
+        c->x_pl = (__nv_bfloat16*)(c->ws + o_xpl);
+        c->h_pl = (__nv_bfloat16*)(c->ws + o_hpl);
+        c->x_sum = (float*)(c->ws + o_xsum);
+        c->h_sum = (float*)(c->ws + o_hsum);
         c->h_ws = (float*)(c->ws + o_h);
         c->y_pairs = (float*)(c->ws + o_y);
         c->x_norm = (__half*)(c->ws + o_xn);
@@ -528,25 +543,35 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
         const int E = g.n_experts, I = g.inter, Is = g.inter_shared;
         // buckets of tau or more pairs go to the tensor cores (tau = 0: none)
         const int tau = c->mma_ok ? c->mma_min_tok : 0;
-        const bool mma_routed = tau > 0 && T >= tau, mma_shared = tau > 0 && T >= tau;
-        const int cap = mma_routed ? tau : 0x7fffffff;
+        const bool mma = tau > 0 && T >= tau;
+        const int cap = mma ? tau : 0x7fffffff;
         const int tiles = (T + kMmaTok - 1) / kMmaTok;
+        const int P = T * (k + 1), hs = c->maxI;
+        __nv_bfloat16 *xh = c->x_pl, *xl = c->x_pl + (size_t)T * H;
+        __nv_bfloat16 *hh = c->h_pl, *hl = c->h_pl + (size_t)P * hs;
         k_group_pairs<<<1, 1024, 0, s>>>(idx, T * k, E, c->e_off, c->plist);
         CKL();
+        if (mma) {
+            const size_t n8 = (size_t)T * H / 8;
+            const unsigned nb = (unsigned)((n8 + 255) / 256 < 1184 ? (n8 + 255) / 256 : 1184);
+            k_split_x<<<nb, 256, 0, s>>>(reinterpret_cast<const uint4*>(xin), n8,
+                                         reinterpret_cast<uint4*>(xh), reinterpret_cast<uint4*>(xl),
+                                         c->x_sum);
+            CKL();
+        }
         k_gateup_grouped<false><<<dim3(I / 16, E), kGrpThreads, grouped_smem_gu(H), s>>>(
             ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
         CKL();
-        if (mma_routed) {
-            k_ffn_mma<false, false><<<dim3(I / 64, E, tiles), kMmaThreads, kMmaSmem, s>>>(
-                ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, tau, g.gelu, c->h_ws, c->maxI,
-                c->y_pairs, c->status);
-            CKL();
-        }
         const int chunks = (T + kGrpChunk - 1) / kGrpChunk;
-        if (mma_shared) {
-            k_ffn_mma<false, true><<<dim3(Is / 64, 1, tiles), kMmaThreads, kMmaSmem, s>>>(
-                ex, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, tau, g.gelu, c->h_ws, c->maxI,
-                c->y_pairs, c->status);
+        const size_t sm_gu = mma_smem_bytes(H), sm_dr = mma_smem_bytes(I), sm_ds = mma_smem_bytes(Is);
+        if (mma) {
+            k_ffn_mma<false, false><<<dim3(I / 64, E, tiles), kMmaThreads, sm_gu, s>>>(
+                ex, stride, sh, H, I, T, k, c->e_off, c->plist, tau, g.gelu, xh, xl, H, c->x_sum,
+                H / 64, hh, hl, hs, c->h_sum, nullptr, c->status);
+            CKL();
+            k_ffn_mma<false, true><<<dim3(Is / 64, 1, tiles), kMmaThreads, sm_gu, s>>>(
+                ex, stride, sh, H, Is, T, k, c->e_off, c->plist, tau, g.gelu, xh, xl, H, c->x_sum,
+                H / 64, hh, hl, hs, c->h_sum, nullptr, c->status);
         } else {
             k_gateup_grouped<true><<<dim3(Is / 16, 1, chunks), kGrpThreads, grouped_smem_gu(H), s>>>(
                 ex, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
@@ -555,16 +580,14 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
         k_down_grouped<false><<<dim3(H / 16, E), kGrpThreads, grouped_smem_dn(I), s>>>(
             ex, stride, sh, H, I, T, c->e_off, c->plist, cap, c->h_ws, c->maxI, c->y_pairs);
         CKL();
-        if (mma_routed) {
-            k_ffn_mma<true, false><<<dim3(H / kMmaRows, E, tiles), kMmaThreads, kMmaSmem, s>>>(
-                ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, tau, g.gelu, c->h_ws, c->maxI,
-                c->y_pairs, c->status);
+        if (mma) {
+            k_ffn_mma<true, false><<<dim3(H / kMmaRows, E, tiles), kMmaThreads, sm_dr, s>>>(
+                ex, stride, sh, H, I, T, k, c->e_off, c->plist, tau, g.gelu, hh, hl, hs, c->h_sum,
+                hs / 64, nullptr, nullptr, 0, nullptr, c->y_pairs, c->status);
             CKL();
-        }
-        if (mma_shared) {
-            k_ffn_mma<true, true><<<dim3(H / kMmaRows, 1, tiles), kMmaThreads, kMmaSmem, s>>>(
-                ex, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, tau, g.gelu, c->h_ws, c->maxI,
-                c->y_pairs, c->status);
+            k_ffn_mma<true, true><<<dim3(H / kMmaRows, 1, tiles), kMmaThreads, sm_ds, s>>>(
+                ex, stride, sh, H, Is, T, k, c->e_off, c->plist, tau, g.gelu, hh, hl, hs, c->h_sum,
+                hs / 64, nullptr, nullptr, 0, nullptr, c->y_pairs, c->status);
         } else {
             k_down_grouped<true><<<dim3(H / 16, 1, chunks), kGrpThreads, grouped_smem_dn(Is), s>>>(
                 ex, stride, sh, H, Is, T, c->e_off, c->plist, cap, c->h_ws, c->maxI, c->y_pairs);

@@ -78,13 +78,15 @@ def test_mma_every_bucket_tiny():
         assert_y_close(y_tc[t], y_cc[t].astype(np.float64), f"tensor vs CUDA cores, token {t}")
 
 
-def test_mma_layer_small_buckets():
-    """Layer shape, threshold 1, T = 8: routed buckets of one or two pairs."""
-    cfg, T = LAYER, 8
+@pytest.mark.parametrize("T,sample", [(8, tuple(range(8))), (200, (0, 63, 64, 130, 199))])
+def test_mma_layer_small_buckets(T, sample):
+    """Layer shape, threshold 1: routed buckets of one or two pairs (T = 8)
+    or about a dozen (T = 200, shared expert in tiles of 64, 64, 64, 8)."""
+    cfg = LAYER
     L = make_layer(cfg, seed=23, bias_std=1.5)
     x = synth.tokens(T, cfg.H, seed=24, device=DEV)
     y, idx = _run(cfg, L, x, T, 1)
-    _check_tokens(cfg, L, x, y, idx, range(T))
+    _check_tokens(cfg, L, x, y, idx, sample)
 
 
 def test_mma_layer_concentrated_buckets():
