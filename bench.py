@@ -85,6 +85,17 @@ def peaks():
     return 6650.0, "fallback"
 
 
+def tensor_peak():
+    """Dense 16-bit tensor peak in TFLOP/s (burst) and where it comes from;
+    fp16 and bf16 share the rate."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 # ------------------------------------------------------------------ clocks --
 class ClockSampler:
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -497,6 +508,7 @@ def run_batched(args):
     dev = torch.device("cuda", 0)
     moeq4.load()
     hbm, kind = peaks()
+    tpk, tkind = tensor_peak()
     copies = [synth.layer_weights(cfg, SEED, l, dev) for l in range(8)]
     objs = [moeq4.Layer.from_dict(d) for d in copies]
     nb, nbs = synth.blob_bytes(cfg.H, cfg.I), synth.blob_bytes(cfg.H, cfg.Is)
@@ -521,15 +533,27 @@ def run_batched(args):
         torch.cuda.synchronize()
         us = e0.elapsed_time(e1) * 1000.0 / reps
         algo = touched * nb + nbs + cfg.E * cfg.H + 2 * cfg.E
+        # useful multiply-adds of the FFNs: gate, up and down of k routed and the shared expert
+        flop = 2.0 * T * 3 * cfg.H * (cfg.k * cfg.I + cfg.Is)
+        if T == 1:
+            path = "fused single-token kernel"
+        elif T >= 32:
+            path = ("tcgen05 kernels (shared expert, buckets of >= 4 pairs) + CUDA-core grouped "
+                    "kernels (smaller buckets)")
+        else:
+            path = "CUDA-core grouped kernels"
         lines.append({"tokens": T, "us_per_step": round(us, 2),
                       "tokens_per_s": round(T / (us * 1e-6), 1),
                       "distinct_experts": round(touched, 1), "algorithmic_bytes": int(algo),
                       "achieved_gbs": round(algo / (us * 1e-6) / 1e9, 1),
                       "frac_of_hbm": round(algo / (us * 1e-6) / 1e9 / hbm, 4),
-                      "path": "fused single-token kernel" if T == 1 else "grouped kernels"})
+                      "ffn_tflops": round(flop / (us * 1e-6) / 1e12, 2),
+                      "frac_of_tensor": round(flop / (us * 1e-6) / 1e12 / tpk, 4),
+                      "path": path})
     moeq4.moe_ctx_check(ctx)
     print(json.dumps({"metric": METRIC, "workload": "batched sweep, one layer", "unit": UNIT,
-                      "peak_gbs": hbm, "peak_kind": kind, "sweep": lines}), flush=True)
+                      "peak_gbs": hbm, "peak_kind": kind, "tensor_peak_tflops": tpk,
+                      "tensor_peak_kind": tkind, "mma_min_tokens": 4, "sweep": lines}), flush=True)
 
 
 def main():

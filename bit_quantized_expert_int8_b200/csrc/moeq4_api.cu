@@ -10,8 +10,10 @@
 #include <string>
 #include <vector>
 
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
-#include "ffn_mma.cuh"
+#include "ffn_tc.cuh"
 #include "ffn_simple.cuh"
 #include "grouped.cuh"
 #include "layer_fused.cuh"
@@ -101,10 +103,10 @@ struct moe_ctx {
     bool grouped_ok = false;           // multi-token steps grouped by expert
     bool mma_ok = false;               // tensor-core kernels usable for this shape
     int mma_min_tok = 0;               // bucket size from which they run (0: never)
-    __nv_bfloat16* x_pl = nullptr;     // [2][maxT][H] x as bf16 hi / lo planes
     __nv_bfloat16* h_pl = nullptr;     // [2][maxT * (k + 1)][maxI] h as bf16 hi / lo planes
-    float* x_sum = nullptr;            // [maxT][H / 64] 64-column group sums of x
     float* h_sum = nullptr;            // [maxT * (k + 1)][maxI / 64] group sums of h
+    __half* xs = nullptr;              // [maxT * (k + 1)][H] x rows: tokens, then pairs by bucket
+    float* xg_sum = nullptr;           // [maxT * (k + 1)][H / 64] their group sums
     int* e_off = nullptr;              // [E + 1] pairs per expert (prefix)
     int* plist = nullptr;              // [maxT * k] pair indices grouped by expert
     uint32_t* dlimb = nullptr;         // packed intermediate of the fused kernel
@@ -165,6 +167,47 @@ extern "C" int moe_ctx_destroy(moe_ctx* c) {
 static size_t grouped_smem_gu(int H) { return (size_t)18 * H + (size_t)kGrpTokens * H * 4; }
 static size_t grouped_smem_dn(int Ie) { return (size_t)9 * Ie + (size_t)kGrpTokens * Ie * 4; }
 
+// cuTensorMapEncodeTiled from the driver (null when unavailable).
+static PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tensor map over the codes of tiled expert blobs: dims {row bytes, rows per
+// tile, tiles, experts}; one copy takes 32 bytes of 128 rows (box_tiles tiles).
+static bool encode_codes(CUtensorMap* m, const void* base, int row_bytes, int rows_per_tile,
+                         size_t tile_stride, int tiles, size_t expert_stride, int experts, int box_tiles) {
+    const cuuint64_t dims[4] = {(cuuint64_t)row_bytes, (cuuint64_t)rows_per_tile, (cuuint64_t)tiles,
+                                (cuuint64_t)experts};
+    const cuuint64_t strides[3] = {(cuuint64_t)row_bytes, (cuuint64_t)tile_stride, (cuuint64_t)expert_stride};
+    const cuuint32_t box[4] = {32u, (cuuint32_t)rows_per_tile, (cuuint32_t)box_tiles, 1u};
+    const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+    return tmap_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box,
+                          es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor map over 16-bit rows: dims {cols, rows, planes}; one copy takes
+// 64 columns x 64 rows of every plane, 128-byte swizzle.
+static bool encode_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int cols, int rows,
+                        int planes) {
+    const cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)planes};
+    const cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)cols * 2 * rows};
+    const cuuint32_t box[3] = {64u, 64u, (cuuint32_t)planes};
+    const cuuint32_t es[3] = {1u, 1u, 1u};
+    return tmap_encoder()(m, dt, 3, const_cast<void*>(base), dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Enables the grouped multi-token path when its tiles fit shared memory.
 static cudaError_t setup_grouped(moe_ctx* c) {
     const MoeConfig& g = c->cfg;
@@ -184,17 +227,17 @@ static cudaError_t setup_grouped(moe_ctx* c) {
         e = cudaFuncSetAttribute(k_down_grouped<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn);
     if (e != cudaSuccess) return e;
     // tensor-core kernels: 4 gate/up tiles (64 indices) or 128 down rows per CTA
-    const size_t sm_gu = mma_smem_bytes(g.hidden), sm_dn = mma_smem_bytes(c->maxI);
-    if (sm_gu > (size_t)optin || sm_dn > (size_t)optin || g.hidden % kMmaRows || g.inter % 64 ||
-        g.inter_shared % 64)
+    const size_t tc_gu = tc_smem_bytes<false>(g.hidden), tc_dn = tc_smem_bytes<true>(c->maxI);
+    if (!tmap_encoder() || tc_gu > (size_t)optin || tc_dn > (size_t)optin || g.hidden % kMmaRows ||
+        g.inter % 64 || g.inter_shared % 64)
         return cudaSuccess;
-    e = cudaFuncSetAttribute(k_ffn_mma<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_gu);
+    e = cudaFuncSetAttribute(k_ffn_tc<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_gu);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_ffn_mma<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_gu);
+        e = cudaFuncSetAttribute(k_ffn_tc<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_gu);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_ffn_mma<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dn);
+        e = cudaFuncSetAttribute(k_ffn_tc<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_dn);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_ffn_mma<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dn);
+        e = cudaFuncSetAttribute(k_ffn_tc<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_dn);
     if (e != cudaSuccess) return e;
     c->mma_ok = true;
     c->mma_min_tok = kMmaDefaultMinTokens;
@@ -281,9 +324,9 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     size_t o_ysh = take(H * sizeof(unsigned long long));
     size_t o_eoff = take((E + 1) * sizeof(int));
     size_t o_plist = take(T * k * sizeof(int));
-    size_t o_xpl = take(2 * T * H * sizeof(__nv_bfloat16));                 // x hi / lo planes
     size_t o_hpl = take(2 * P * (size_t)c->maxI * sizeof(__nv_bfloat16));   // h hi / lo planes
-    size_t o_xsum = take(T * (H / 64) * sizeof(float));                      // x group sums
+    size_t o_xs = take(P * H * sizeof(__half));                              // x rows, bucket order
+    size_t o_xgsum = take(P * (H / 64) * sizeof(float));                     // their group sums
     size_t o_hsum = take(P * (size_t)(c->maxI / 64) * sizeof(float));        // h group sums
     int n_sms_dev = 0;
     cudaDeviceGetAttribute(&n_sms_dev, cudaDevAttrMultiProcessorCount, c->device);
@@ -299,9 +342,9 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
         c->pairs = (MoeFfnPair*)(c->ws + o_pairs);
         c->e_off = (int*)(c->ws + o_eoff);
         c->plist = (int*)(c->ws + o_plist);
-        c->x_pl = (__nv_bfloat16*)(c->ws + o_xpl);
         c->h_pl = (__nv_bfloat16*)(c->ws + o_hpl);
-        c->x_sum = (float*)(c->ws + o_xsum);
+        c->xs = (__half*)(c->ws + o_xs);
+        c->xg_sum = (float*)(c->ws + o_xgsum);
         c->h_sum = (float*)(c->ws + o_hsum);
         c->h_ws = (float*)(c->ws + o_h);
         c->y_pairs = (float*)(c->ws + o_y);
@@ -541,37 +584,56 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
         const uint8_t* ex = static_cast<const uint8_t*>(L->experts);
         const uint8_t* sh = static_cast<const uint8_t*>(L->shared_blob);
         const int E = g.n_experts, I = g.inter, Is = g.inter_shared;
-        // buckets of tau or more pairs go to the tensor cores (tau = 0: none)
+        // In steps of at least kMmaMinStep tokens, routed buckets of tau or more
+        // pairs and the shared expert (T >= tau) run on the tensor cores
+        // (tau = 0: none); the rest on the CUDA-core grouped kernels.
         const int tau = c->mma_ok ? c->mma_min_tok : 0;
-        const bool mma = tau > 0 && T >= tau;
-        const int cap = mma ? tau : 0x7fffffff;
+        const bool tc = tau > 0 && T >= kMmaMinStep;
+        const bool tc_shared = tc && T >= tau;
+        const int cap = tc ? tau : 0x7fffffff;
         const int tiles = (T + kMmaTok - 1) / kMmaTok;
         const int P = T * (k + 1), hs = c->maxI;
-        __nv_bfloat16 *xh = c->x_pl, *xl = c->x_pl + (size_t)T * H;
         __nv_bfloat16 *hh = c->h_pl, *hl = c->h_pl + (size_t)P * hs;
         k_group_pairs<<<1, 1024, 0, s>>>(idx, T * k, E, c->e_off, c->plist);
         CKL();
-        if (mma) {
-            const size_t n8 = (size_t)T * H / 8;
-            const unsigned nb = (unsigned)((n8 + 255) / 256 < 1184 ? (n8 + 255) / 256 : 1184);
-            k_split_x<<<nb, 256, 0, s>>>(reinterpret_cast<const uint4*>(xin), n8,
-                                         reinterpret_cast<uint4*>(xh), reinterpret_cast<uint4*>(xl),
-                                         c->x_sum);
+        CUtensorMap m_cgr, m_cgs, m_cdr, m_cds, m_x, m_h;
+        TcArgs ta{};
+        if (tc) {
+            // x rows in bucket order (tokens first) with their group sums; this call's tensor maps
+            k_gather_x<<<dim3((H + 2047) / 2048, P < 65535 ? P : 65535), 256, 0, s>>>(
+                xin, H, T, k, P, c->plist, c->xs, c->xg_sum);
             CKL();
+            const BlobLayout Lr(H, I), Ls(H, Is);
+            const size_t sb = Ls.bytes;
+            if (!encode_codes(&m_cgr, ex, H / 2, 32, Lr.gu_tile, I / 16, stride, E, 4) ||
+                !encode_codes(&m_cgs, sh, H / 2, 32, Ls.gu_tile, Is / 16, sb, 1, 4) ||
+                !encode_codes(&m_cdr, ex + Lr.dn_base, I / 2, 16, Lr.dn_tile, H / 16, stride, E, 8) ||
+                !encode_codes(&m_cds, sh + Ls.dn_base, Is / 2, 16, Ls.dn_tile, H / 16, sb, 1, 8) ||
+                !encode_rows(&m_x, c->xs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, H, P, 1) ||
+                !encode_rows(&m_h, hh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hs, P, 2))
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+            ta.H = H; ta.T = T; ta.k = k; ta.min_tok = tau; ta.gelu = g.gelu;
+            ta.e_off = c->e_off; ta.list = c->plist;
+            ta.h_hi = hh; ta.h_lo = hl; ta.h_sum = c->h_sum; ta.hs = hs;
+            ta.y_pairs = c->y_pairs; ta.status = c->status;
         }
+        const int chunks = (T + kGrpChunk - 1) / kGrpChunk;
         k_gateup_grouped<false><<<dim3(I / 16, E), kGrpThreads, grouped_smem_gu(H), s>>>(
             ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
         CKL();
-        const int chunks = (T + kGrpChunk - 1) / kGrpChunk;
-        const size_t sm_gu = mma_smem_bytes(H), sm_dr = mma_smem_bytes(I), sm_ds = mma_smem_bytes(Is);
-        if (mma) {
-            k_ffn_mma<false, false><<<dim3(I / 64, E, tiles), kMmaThreads, sm_gu, s>>>(
-                ex, stride, sh, H, I, T, k, c->e_off, c->plist, tau, g.gelu, xh, xl, H, c->x_sum,
-                H / 64, hh, hl, hs, c->h_sum, nullptr, c->status);
+        TcArgs gu = ta;
+        gu.b_sum = c->xg_sum;
+        gu.bs_stride = H / 64;
+        if (tc) {
+            gu.Ie = I;
+            k_ffn_tc<false, false><<<dim3(I / 64, E, tiles), kTcThreads, tc_smem_bytes<false>(H), s>>>(
+                m_cgr, m_x, ex, stride, sh, gu);
             CKL();
-            k_ffn_mma<false, true><<<dim3(Is / 64, 1, tiles), kMmaThreads, sm_gu, s>>>(
-                ex, stride, sh, H, Is, T, k, c->e_off, c->plist, tau, g.gelu, xh, xl, H, c->x_sum,
-                H / 64, hh, hl, hs, c->h_sum, nullptr, c->status);
+        }
+        if (tc_shared) {
+            gu.Ie = Is;
+            k_ffn_tc<false, true><<<dim3(Is / 64, 1, tiles), kTcThreads, tc_smem_bytes<false>(H), s>>>(
+                m_cgs, m_x, ex, stride, sh, gu);
         } else {
             k_gateup_grouped<true><<<dim3(Is / 16, 1, chunks), kGrpThreads, grouped_smem_gu(H), s>>>(
                 ex, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
@@ -580,14 +642,19 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
         k_down_grouped<false><<<dim3(H / 16, E), kGrpThreads, grouped_smem_dn(I), s>>>(
             ex, stride, sh, H, I, T, c->e_off, c->plist, cap, c->h_ws, c->maxI, c->y_pairs);
         CKL();
-        if (mma) {
-            k_ffn_mma<true, false><<<dim3(H / kMmaRows, E, tiles), kMmaThreads, sm_dr, s>>>(
-                ex, stride, sh, H, I, T, k, c->e_off, c->plist, tau, g.gelu, hh, hl, hs, c->h_sum,
-                hs / 64, nullptr, nullptr, 0, nullptr, c->y_pairs, c->status);
+        TcArgs dn = ta;
+        dn.b_sum = c->h_sum;
+        dn.bs_stride = hs / 64;
+        if (tc) {
+            dn.Ie = I;
+            k_ffn_tc<true, false><<<dim3(H / kMmaRows, E, tiles), kTcThreads, tc_smem_bytes<true>(I), s>>>(
+                m_cdr, m_h, ex, stride, sh, dn);
             CKL();
-            k_ffn_mma<true, true><<<dim3(H / kMmaRows, 1, tiles), kMmaThreads, sm_ds, s>>>(
-                ex, stride, sh, H, Is, T, k, c->e_off, c->plist, tau, g.gelu, hh, hl, hs, c->h_sum,
-                hs / 64, nullptr, nullptr, 0, nullptr, c->y_pairs, c->status);
+        }
+        if (tc_shared) {
+            dn.Ie = Is;
+            k_ffn_tc<true, true><<<dim3(H / kMmaRows, 1, tiles), kTcThreads, tc_smem_bytes<true>(Is), s>>>(
+                m_cds, m_h, ex, stride, sh, dn);
         } else {
             k_down_grouped<true><<<dim3(H / 16, 1, chunks), kGrpThreads, grouped_smem_dn(Is), s>>>(
                 ex, stride, sh, H, Is, T, c->e_off, c->plist, cap, c->h_ws, c->maxI, c->y_pairs);
