@@ -47,6 +47,8 @@ def parse():
     p.add_argument("--tokens", type=int, default=N_TOKENS)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
+    p.add_argument("--batch-sizes", default="1,8,32,64,128,256",
+                   help="tokens per step of the batched sweep (comma-separated)")
     p.add_argument("--workload", choices=("stack", "streaming", "batched"), default="stack",
                    help="stack (default, the headline line), streaming (experts in pinned host "
                         "memory behind the LFU cache) or batched (one layer, T tokens per step)")
@@ -512,9 +514,10 @@ def run_batched(args):
     copies = [synth.layer_weights(cfg, SEED, l, dev) for l in range(8)]
     objs = [moeq4.Layer.from_dict(d) for d in copies]
     nb, nbs = synth.blob_bytes(cfg.H, cfg.I), synth.blob_bytes(cfg.H, cfg.Is)
-    ctx = moeq4.Context(cfg, 256)
+    sizes = [int(v) for v in args.batch_sizes.split(",")]
+    ctx = moeq4.Context(cfg, max(sizes))
     lines = []
-    for T in (1, 8, 32, 64, 128, 256):
+    for T in sizes:
         x = synth.tokens(T, cfg.H, SEED + 3, dev)
         y = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
         idx = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
