@@ -498,6 +498,18 @@ def run_streaming(args):
         "h2d_link_gbs_measured": round(link, 2)}), flush=True)
 
 
+def bucket_split(counts, T, min_tokens=4, min_step=32):
+    """Experts of one step by the kernel that serves them: `counts` holds the
+    pairs routed to each expert.  In steps of at least `min_step` tokens a
+    bucket of `min_tokens` or more pairs runs on tcgen05; every other used
+    expert on the CUDA-core grouped kernels.  Returns (tcgen05, grouped)."""
+    used = [c for c in counts if c > 0]
+    if T < min_step or min_tokens <= 0:
+        return 0, len(used)
+    tc = sum(1 for c in used if c >= min_tokens)
+    return tc, len(used) - tc
+
+
 def run_batched(args):
     """Batched decode: one layer of the stack configuration (no router bias,
     independent routings) at T tokens per step; 8 weight copies rotated so the
@@ -522,9 +534,15 @@ def run_batched(args):
         y = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
         idx = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
         touched = 0
+        n_tc = n_grp = 0
         for o in objs:
             moeq4.moe_layer_decode(ctx, o, x, T, y, idx)
             touched += torch.unique(idx).numel()
+            if T > 1:
+                counts = torch.bincount(idx.flatten().long(), minlength=cfg.E).tolist()
+                a, b = bucket_split(counts, T)
+                n_tc += a
+                n_grp += b
         touched /= len(objs)
         reps = max(8, min(400, int(4000 / T)))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -552,6 +570,11 @@ def run_batched(args):
                       "frac_of_hbm": round(algo / (us * 1e-6) / 1e9 / hbm, 4),
                       "ffn_tflops": round(flop / (us * 1e-6) / 1e12, 2),
                       "frac_of_tensor": round(flop / (us * 1e-6) / 1e12 / tpk, 4),
+                      # max(bytes / HBM peak, flops / tensor peak) over the measured time
+                      "frac_of_roofline": round(max(algo / (hbm * 1e9), flop / (tpk * 1e12)) /
+                                                (us * 1e-6), 4),
+                      "experts_tcgen05": round(n_tc / len(objs), 1),
+                      "experts_grouped": round(n_grp / len(objs), 1),
                       "path": path})
     moeq4.moe_ctx_check(ctx)
     print(json.dumps({"metric": METRIC, "workload": "batched sweep, one layer", "unit": UNIT,
