@@ -1,0 +1,106 @@
+"""CPU pins of the arithmetic the tensor-core FFN kernels rely on.
+
+The kernels never round a weight.  The raw 4-bit codes enter the MMA as
+exact 16-bit integers, and each 64-column group is folded as
+s_g * P_g + b_g * S_g, with P_g = sum q x and S_g = sum x.  x (fp16) enters
+exactly; h (fp32) enters as two bf16 planes hi + lo.  These tests check each
+claim with numpy/torch on the CPU, and the whole gate/up step against the
+oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_quantized_expert_int8_b200 import synth
+
+G = 64
+
+
+def _unpack(words):
+    """int32 words [R, K/8] (low nibble first) -> codes [R, K]."""
+    w = words.numpy().astype(np.int64) & 0xFFFFFFFF
+    shifts = np.arange(8) * 4
+    return ((w[:, :, None] >> shifts) & 15).reshape(w.shape[0], -1)
+
+
+def _quantised(R, K, seed):
+    w = synth.randn((R, K), seed, "cpu", synth.WEIGHT_STD)
+    words, s16, b16 = synth.quantize_q4(w)
+    return _unpack(words), s16.double().numpy(), b16.double().numpy()
+
+
+def test_group_fold_equals_dequantised_product():
+    """sum_g (s_g P_g + b_g S_g) is the product with w = s q + b (fp64)."""
+    R, K, T = 48, 256, 5
+    q, s, b = _quantised(R, K, 101)
+    x = synth.tokens(T, K, seed=102).double().numpy()
+    w = (q.reshape(R, K // G, G) * s[..., None] + b[..., None]).reshape(R, K)
+    ref = w @ x.T
+    qg = q.reshape(R, K // G, G).astype(np.float64)
+    xg = x.reshape(T, K // G, G)
+    P = np.einsum("rgc,tgc->rgt", qg, xg)             # per-group code products
+    S = xg.sum(-1).T                                  # [groups, T]
+    fold = (s[..., None] * P + b[..., None] * S[None]).sum(1)
+    np.testing.assert_allclose(fold, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_codes_exact_in_both_16_bit_operand_types():
+    """0..15 are exact in fp16 and bf16, and the mantissa constructions the
+    converters use (0x6400 | q = 1024 + q in fp16, 0x4300 | q = 128 + q in
+    bf16) give them exactly."""
+    q = np.arange(16, dtype=np.uint16)
+    f16 = (np.uint16(0x6400) | q).view(np.float16).astype(np.float64) - 1024.0
+    bf = torch.from_numpy((np.uint16(0x4300) | q).astype(np.int16)).view(torch.bfloat16)
+    assert np.array_equal(f16, q.astype(np.float64))
+    assert np.array_equal(bf.double().numpy() - 128.0, q.astype(np.float64))
+    assert np.array_equal(torch.from_numpy(q.astype(np.float32)).to(torch.bfloat16).double().numpy(),
+                          q.astype(np.float64))
+
+
+def test_fp16_is_exact_as_bf16_hi_plus_lo():
+    """Every finite fp16 value equals bf16(v) + bf16(v - bf16(v))."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    v = bits.view(np.float16)
+    v = v[np.isfinite(v)].astype(np.float32)
+    t = torch.from_numpy(v)
+    hi = t.to(torch.bfloat16).float()
+    lo = (t - hi).to(torch.bfloat16).float()
+    assert torch.equal((hi.double() + lo.double()), t.double())
+
+
+@pytest.mark.parametrize("scale", [1e-6, 1e-2, 1.0, 1e3, 6e4])
+def test_bf16_hi_lo_split_relative_error(scale):
+    """h = hi + lo to within 2^-16 of |h| (bf16 keeps 8 significant bits per
+    term), over several magnitudes."""
+    g = torch.Generator().manual_seed(7)
+    h = torch.randn(100000, generator=g) * scale
+    hi = h.to(torch.bfloat16).float()
+    lo = (h - hi).to(torch.bfloat16).float()
+    err = (h.double() - hi.double() - lo.double()).abs()
+    assert (err <= h.double().abs() * 2.0 ** -16).all()
+
+
+def test_gateup_fold_matches_oracle():
+    """The tensor-core gate/up arithmetic (exact codes and fp16 x, fp32 group
+    sums, fold s P + b S in fp32, GELU(gate) * up) against the oracle's h for
+    one expert blob; tolerance of an fp32 computation."""
+    H, I = 256, 128
+    blob = synth.expert_blob(H, I, seed=31)
+    x16 = synth.tokens(1, H, seed=32)[0]
+    _, h_ref = oracle.expert_ffn(blob.numpy(), H, I, x16.double().numpy())
+    # rebuild gate and up as the kernels see them: quantise the same draws
+    w_gu = synth.randn((2 * I, H), synth.seed_for(31, 0), "cpu", synth.WEIGHT_STD)
+    words, s16, b16 = synth.quantize_q4(w_gu)
+    q = _unpack(words).astype(np.float32)
+    s, b = s16.float().numpy(), b16.float().numpy()
+    x = x16.float().numpy()
+    qg = q.reshape(2 * I, H // G, G)
+    xg = x.reshape(H // G, G)
+    P = (qg * xg[None]).sum(-1, dtype=np.float32)     # exact products, fp32 sums
+    S = xg.sum(-1, dtype=np.float32)
+    D = (s * P + b * S[None]).sum(-1, dtype=np.float32)
+    gate, up = D[:I].astype(np.float64), D[I:].astype(np.float64)
+    h = np.array([oracle.gelu(g_) for g_ in gate]) * up
+    rel = np.linalg.norm(h - h_ref) / np.linalg.norm(h_ref)
+    assert rel < 1e-5, rel
