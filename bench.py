@@ -35,6 +35,7 @@ N_LAYERS = 30
 N_TOKENS = 256
 SEED = 0
 BIAS_STD = 1.5
+REPEATS = 5          # timed runs per step size of the batched sweep (median reported)
 
 
 def parse():
@@ -307,25 +308,28 @@ def roofline(ctx, layers, cfg, dev, stream):
     from bit_quantized_expert_int8_b200 import moeq4, synth
     hbm, kind = peaks()
     n = len(layers)
-    x = synth.tokens(1, cfg.H, SEED + 77, dev)
+    reps = 20
+    # a distinct token for every launch of the graph, so no launch can profit
+    # from the routing (or the weights) of an earlier replay
+    xs = synth.tokens(n * reps, cfg.H, SEED + 77, dev)
     y = torch.empty((1, cfg.H), dtype=torch.float32, device=dev)
     objs = [moeq4.Layer.from_dict(d) for d in layers]
     side = torch.cuda.Stream()
     side.wait_stream(stream)
     with torch.cuda.stream(side):
-        for o in objs:                                        # warm up
-            moeq4.moe_layer_decode(ctx, o, x, 1, y, stream=side)
+        for i, o in enumerate(objs):                          # warm up
+            moeq4.moe_layer_decode(ctx, o, xs[i:i + 1], 1, y, stream=side)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=side):
-            for o in objs:
-                moeq4.moe_layer_decode(ctx, o, x, 1, y, stream=side)
-        reps = 20
-        for _ in range(3):
+            for r in range(reps):
+                for i, o in enumerate(objs):
+                    j = r * n + i
+                    moeq4.moe_layer_decode(ctx, o, xs[j:j + 1], 1, y, stream=side)
+        for _ in range(2):
             g.replay()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(side)
-        for _ in range(reps):
-            g.replay()
+        g.replay()
         e1.record(side)
     torch.cuda.synchronize()
     moeq4.moe_ctx_check(ctx)
@@ -463,19 +467,22 @@ def run_streaming(args):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     hits = misses = 0
-    ms = 0.0
+    times = []
+    clocks = ClockSampler(0)
+    clocks.start()
     for _ in range(args.steps):
         e0.record()
         step()
         e1.record()
         torch.cuda.synchronize()
-        ms += e0.elapsed_time(e1)
+        times.append(e0.elapsed_time(e1))
         for (_, _, _, table) in keep:
             tb = moeq4.read_lfu_table(table)
             hits += tb.hits
             misses += tb.misses
+    clk = clocks.stop()
     moeq4.moe_ctx_check(ctx)
-    ms /= args.steps
+    ms = statistics.median(times)
     h2d = misses / args.steps * nb
     # the link itself: one pinned host -> device copy of 1 GiB
     src = torch.empty(1 << 30, dtype=torch.uint8, pin_memory=True)
@@ -490,9 +497,12 @@ def run_streaming(args):
     print(json.dumps({
         "metric": METRIC, "workload": f"streaming{L}x{T}", "value": round(T / (ms / 1000.0), 3),
         "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "ms_per_step": round(ms, 3), "ms_per_step_min_max": [round(min(times), 3),
+                                                              round(max(times), 3)],
+        "timing": f"median of {len(times)} steps", "higher_is_better": True,
         "config": {"layers": L, "tokens": T, "slots": cfg.S, "cache": "cold at each step",
                    "expert_store": "pinned host memory"},
+        "clocks": clk,
         "hit_rate": round(hits / max(1, hits + misses), 4),
         "h2d_bytes_per_step": int(h2d), "h2d_gbs_over_step": round(h2d / (ms * 1e-3) / 1e9, 2),
         "h2d_link_gbs_measured": round(link, 2)}), flush=True)
@@ -529,6 +539,8 @@ def run_batched(args):
     sizes = [int(v) for v in args.batch_sizes.split(",")]
     ctx = moeq4.Context(cfg, max(sizes))
     lines = []
+    clocks = ClockSampler(0)
+    clocks.start()
     for T in sizes:
         x = synth.tokens(T, cfg.H, SEED + 3, dev)
         y = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
@@ -546,13 +558,16 @@ def run_batched(args):
         touched /= len(objs)
         reps = max(8, min(400, int(4000 / T)))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        e0.record()
-        for r in range(reps):
-            moeq4.moe_layer_decode(ctx, objs[r % len(objs)], x, T, y)
-        e1.record()
-        torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1000.0 / reps
+        runs = []
+        for _ in range(REPEATS):
+            torch.cuda.synchronize()
+            e0.record()
+            for r in range(reps):
+                moeq4.moe_layer_decode(ctx, objs[r % len(objs)], x, T, y)
+            e1.record()
+            torch.cuda.synchronize()
+            runs.append(e0.elapsed_time(e1) * 1000.0 / reps)
+        us = statistics.median(runs)
         algo = touched * nb + nbs + cfg.E * cfg.H + 2 * cfg.E
         # useful multiply-adds of the FFNs: gate, up and down of k routed and the shared expert
         flop = 2.0 * T * 3 * cfg.H * (cfg.k * cfg.I + cfg.Is)
@@ -564,6 +579,7 @@ def run_batched(args):
         else:
             path = "CUDA-core grouped kernels"
         lines.append({"tokens": T, "us_per_step": round(us, 2),
+                      "us_min_max": [round(min(runs), 2), round(max(runs), 2)],
                       "tokens_per_s": round(T / (us * 1e-6), 1),
                       "distinct_experts": round(touched, 1), "algorithmic_bytes": int(algo),
                       "achieved_gbs": round(algo / (us * 1e-6) / 1e9, 1),
@@ -576,8 +592,10 @@ def run_batched(args):
                       "experts_tcgen05": round(n_tc / len(objs), 1),
                       "experts_grouped": round(n_grp / len(objs), 1),
                       "path": path})
+    clk = clocks.stop()
     moeq4.moe_ctx_check(ctx)
     print(json.dumps({"metric": METRIC, "workload": "batched sweep, one layer", "unit": UNIT,
+                      "timing": f"median of {REPEATS} runs of each step size", "clocks": clk,
                       "peak_gbs": hbm, "peak_kind": kind, "tensor_peak_tflops": tpk,
                       "tensor_peak_kind": tkind, "mma_min_tokens": 4, "sweep": lines}), flush=True)
 

@@ -121,6 +121,22 @@ struct moe_ctx {
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Raises a kernel's dynamic shared-memory limit to at least `bytes`.  The
+// attribute belongs to the function and holds for the whole process, so it is
+// never lowered: a context created later for a smaller shape must not shrink
+// the limit under a larger context that is still in use.
+static std::mutex g_smem_attr_mu;
+
+template <typename F>
+static cudaError_t raise_smem(F* fn, size_t bytes) {
+    std::lock_guard<std::mutex> lock(g_smem_attr_mu);
+    cudaFuncAttributes fa{};
+    cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+    if (e != cudaSuccess) return e;
+    if ((size_t)fa.maxDynamicSharedSizeBytes >= bytes) return cudaSuccess;
+    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
 static int check_cfg(const MoeConfig* c) {
     if (!c) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
     if (c->hidden <= 0 || c->hidden % MOE_GROUP || c->inter <= 0 || c->inter % MOE_GROUP ||
@@ -218,26 +234,26 @@ static cudaError_t setup_grouped(moe_ctx* c) {
     const size_t dn = grouped_smem_dn(c->maxI);
     c->grouped_ok = gu <= (size_t)optin && dn <= (size_t)optin;
     if (!c->grouped_ok) return cudaSuccess;
-    e = cudaFuncSetAttribute(k_gateup_grouped<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gu);
+    e = raise_smem(k_gateup_grouped<false>, (int)gu);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_gateup_grouped<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gu);
+        e = raise_smem(k_gateup_grouped<true>, (int)gu);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_down_grouped<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn);
+        e = raise_smem(k_down_grouped<false>, (int)dn);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_down_grouped<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn);
+        e = raise_smem(k_down_grouped<true>, (int)dn);
     if (e != cudaSuccess) return e;
     // tensor-core kernels: 4 gate/up tiles (64 indices) or 128 down rows per CTA
     const size_t tc_gu = tc_smem_bytes<false>(g.hidden), tc_dn = tc_smem_bytes<true>(c->maxI);
     if (!tmap_encoder() || tc_gu > (size_t)optin || tc_dn > (size_t)optin || g.hidden % kMmaRows ||
         g.inter % 64 || g.inter_shared % 64)
         return cudaSuccess;
-    e = cudaFuncSetAttribute(k_ffn_tc<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_gu);
+    e = raise_smem(k_ffn_tc<false, false>, (size_t)tc_gu);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_ffn_tc<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_gu);
+        e = raise_smem(k_ffn_tc<false, true>, (size_t)tc_gu);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_ffn_tc<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_dn);
+        e = raise_smem(k_ffn_tc<true, false>, (size_t)tc_dn);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_ffn_tc<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_dn);
+        e = raise_smem(k_ffn_tc<true, true>, (size_t)tc_dn);
     if (e != cudaSuccess) return e;
     c->mma_ok = true;
     c->mma_min_tok = kMmaDefaultMinTokens;
@@ -286,8 +302,7 @@ static cudaError_t setup_fused(moe_ctx* c) {
     c->f_stages = ns;
     c->f_stage_bytes = (int)stage;
     c->f_smem = (size_t)ns * stage + fused_fixed_smem(g.hidden, NCr, NCs, ns);
-    return cudaFuncSetAttribute(c->f_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)c->f_smem);
+    return raise_smem(c->f_kernel, (int)c->f_smem);
 }
 
 extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** out) {
@@ -372,13 +387,11 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking);
     const int smem_router = (int)(H * sizeof(long long));
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_router);
+        e = raise_smem(k_router, smem_router);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_ffn_gateup_simple, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(H * sizeof(float)));
+        e = raise_smem(k_ffn_gateup_simple, (int)(H * sizeof(float)));
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_ffn_down_simple, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(c->maxI * sizeof(float)));
+        e = raise_smem(k_ffn_down_simple, (int)(c->maxI * sizeof(float)));
     if (e == cudaSuccess) e = setup_grouped(c);
     if (e == cudaSuccess) e = setup_fused(c);
     if (e != cudaSuccess) {
@@ -913,7 +926,10 @@ static std::mutex g_noalloc_mu;
 static void* g_noalloc_dev_ptr[kNoAllocMaxDevices];      // per device ordinal
 
 // Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and remembered.
+// per device (with that device current) and remembered, together with the
+// router kernel's shared-memory limit.  A cudaDeviceReset unloads the module
+// and invalidates the remembered address: the entry point must not be used
+// after one.
 static int noalloc_scratch(unsigned char** out) {
     int dev = -1;
     CK(cudaGetDevice(&dev));
@@ -927,6 +943,12 @@ static int noalloc_scratch(unsigned char** out) {
         if (e != cudaSuccess || !p)
             return fail(MOE_ERR_CUDA, "moe_router_topk_noalloc: cudaGetSymbolAddress: %s",
                         cudaGetErrorString(e));
+        // k_router takes hidden * 8 bytes of dynamic shared memory; allow the
+        // largest hidden this entry point accepts, whatever contexts exist
+        const cudaError_t ea = raise_smem(k_router, (size_t)kNoAllocMaxHidden * sizeof(long long));
+        if (ea != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "moe_router_topk_noalloc: shared-memory limit: %s",
+                        cudaGetErrorString(ea));
         g_noalloc_dev_ptr[dev] = p;
     }
     *out = static_cast<unsigned char*>(g_noalloc_dev_ptr[dev]);

@@ -184,3 +184,42 @@ def routing_sequence(T: int, E: int, k: int, seed: int, zipf: float = 1.1):
     rows = torch.multinomial(w.expand(T, E), k, replacement=False,
                              generator=g)
     return rows.to(torch.int32)
+
+
+# ------------------------------------------------------- hard activations --
+# Token rows for edge-case parity tests: magnitudes and shapes that the N(0, 1)
+# workload never produces.  Like everything here they are plain seeded data.
+
+def outlier_tokens(T: int, H: int, seed: int, device="cpu", factor: float = 1000.0,
+                   every: int = 4, offset: int = 17):
+    """N(0, 1) rows in which channel `offset` of every `every`-th 64-column
+    group is `factor` times larger: groups whose one channel dwarfs the other
+    63 (outlier channels), rounded to fp16."""
+    x = randn((T, H), seed_for(seed, ROLE_TOKENS, 101), device, 1.0)
+    ch = torch.arange(offset, H, GROUP * every, device=device)
+    x[:, ch] *= factor
+    return x.clamp(-65504.0, 65504.0).to(torch.float16)
+
+
+def student_t_tokens(T: int, H: int, seed: int, device="cpu", df: int = 3):
+    """Heavy-tailed rows: Student-t with `df` degrees of freedom,
+    z / sqrt(chi2_df / df) from seeded normals, rounded to fp16."""
+    z = randn((T, H), seed_for(seed, ROLE_TOKENS, 102), device, 1.0)
+    c = randn((df, T, H), seed_for(seed, ROLE_TOKENS, 103), device, 1.0)
+    t = z / torch.sqrt((c * c).sum(0) / df)
+    return t.clamp(-65504.0, 65504.0).to(torch.float16)
+
+
+def extreme_tokens(T: int, H: int, seed: int, device="cpu"):
+    """N(0, 1) rows with, at seeded positions of every row, the fp16 extremes:
+    +-65504, the smallest subnormal (+-2^-24), the largest subnormal
+    (1023 * 2^-24), a mid subnormal, and zeros (including -0)."""
+    x = randn((T, H), seed_for(seed, ROLE_TOKENS, 104), device, 1.0).to(torch.float16)
+    specials = torch.tensor([65504.0, -65504.0, 2.0 ** -24, -(2.0 ** -24), 1023 * 2.0 ** -24,
+                             -(517 * 2.0 ** -24), 0.0, -0.0], dtype=torch.float16)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed_for(seed, ROLE_TOKENS, 105))
+    for t in range(T):
+        pos = torch.randperm(H, generator=g)[:3 * specials.numel()]
+        x[t, pos.to(device)] = specials.repeat(3).to(device)
+    return x

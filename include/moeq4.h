@@ -164,7 +164,11 @@ const char *moe_last_error(void);
  * (8-bit router: [LH] pipeline step 1; [DS] item 1).
  */
 
-/* Size in bytes of one expert blob with the given hidden/intermediate. */
+/* Size in bytes of one expert blob with the given hidden/intermediate: the
+ * unit an expert cache fill copies ([DS] "Trois optimisations cles" item 3;
+ * [DT] "Wat is de belangrijkste architectuurtruuc": only the selected
+ * experts' weights are brought in).  Returns 0 when hidden or inter is not a
+ * positive multiple of 64. */
 size_t moe_blob_bytes(int hidden, int inter);
 
 /* ---------------------------------------------------------- router ----
@@ -204,9 +208,11 @@ int moe_router_topk(moe_ctx *ctx, const int8_t *Wr, const moe_half *row_scale,
  * and <= 6144; larger requests return MOE_ERR_UNSUPPORTED_SHAPE before any
  * CUDA call.  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress, with that device current); make that first
- * call before any stream capture.  Every call on a device shares the one
- * array: calls whose executions overlap on the GPU (other streams, other
- * host threads) race on it and must be serialised by the caller. */
+ * call before any stream capture.  The address is remembered for the life of
+ * the process: after a cudaDeviceReset this entry point must not be called.
+ * Every call on a device shares the one array: calls whose executions overlap
+ * on the GPU (other streams, other host threads) race on it and must be
+ * serialised by the caller. */
 int moe_router_topk_noalloc(int n_experts, int hidden, int top_k, int renorm,
                             const int8_t *Wr, const moe_half *row_scale,
                             const float *bias, const moe_half *x, int T,
@@ -214,6 +220,10 @@ int moe_router_topk_noalloc(int n_experts, int hidden, int top_k, int renorm,
                             moe_stream_t stream);
 
 /* ----------------------------------------------------- expert FFN ----
+ * The expert feed-forward block on 4-bit "MLX affine" weights ([RM]
+ * "L'affirmation des 2 Go ...": routed and shared experts stored as 4-bit
+ * affine groups; [DT] "Wat is de belangrijkste architectuurtruuc": each
+ * token runs the shared expert and its selected experts).
  * Grouped expert FFN over n_pairs (expert, token) pairs: for pair p,
  *   g = Wg x, u = Wu x, h = GELU(g) * u, y[p] = Wd h,
  * with x = row pairs[p].token of x, weights dequantised from the pair's

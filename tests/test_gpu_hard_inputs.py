@@ -1,0 +1,104 @@
+"""Parity on activations the N(0, 1) workload never produces, at the layer
+shape (hidden 2816, 128 experts, top-8), for the three kernels that serve a
+layer: the fused single-token kernel (T = 1), the CUDA-core grouped kernels
+(T = 8) and the tensor-core kernels (T = 40 with every bucket on tcgen05).
+
+Cases (rows from the seeded generators in synth):
+- outlier channels: one channel of every fourth 64-column group is 1000x the
+  other 63, fed raw and through the RMSNorm prologue;
+- Student-t (3 degrees of freedom) heavy tails, raw and through RMSNorm;
+- fp16 extremes (+-65504, smallest and largest subnormals, zeros) fed raw:
+  the router must stay bit-exact; the FFN output is then of size 1e5 and up,
+  where the absolute bound scales with max |y| (gpu_util).
+
+Routing (indices) is compared bit for bit, weights within the router tests'
+tolerance, y within rel L2 <= 1e-3 and max abs <= 2e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_quantized_expert_int8_b200 import build, moeq4, synth
+from bit_quantized_expert_int8_b200.config import LAYER
+from gpu_util import assert_y_close, assert_y_close_scaled, make_layer, np_layer, np_of
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+CFG = LAYER
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    moeq4.load()
+    assert torch.cuda.is_available()
+    yield
+    torch.cuda.synchronize()
+
+
+@pytest.fixture(scope="module")
+def layer():
+    L = make_layer(CFG, seed=61, bias_std=1.5)
+    return L, np_layer(L), moeq4.Layer.from_dict(L)
+
+
+def _rows(case, T, seed):
+    if case.startswith("outlier"):
+        return synth.outlier_tokens(T, CFG.H, seed, DEV)
+    if case.startswith("student"):
+        return synth.student_t_tokens(T, CFG.H, seed, DEV)
+    return synth.extreme_tokens(T, CFG.H, seed, DEV)
+
+
+CASES = ["outlier_raw", "outlier_prenorm", "student_raw", "student_prenorm", "extreme_raw"]
+PATHS = [(1, None, (0,)), (8, 0, (0, 5, 7)), (40, 1, (0, 17, 39))]   # (T, mma threshold, tokens)
+
+
+@pytest.mark.parametrize("case", CASES)
+@pytest.mark.parametrize("T,tau,sample", PATHS)
+def test_hard_activations(layer, case, T, tau, sample):
+    L, Ln, lay = layer
+    prenorm = case.endswith("prenorm")
+    x = _rows(case, T, seed=70 + T)
+    x0 = np_of(x).copy()
+    ctx = moeq4.Context(CFG, T)
+    if tau is not None:
+        moeq4.moe_set_mma_min_tokens(ctx, tau)
+    y = torch.empty((T, CFG.H), device=DEV)
+    idx = torch.empty((T, CFG.k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, CFG.k), device=DEV)
+    xn = torch.empty((T, CFG.H), dtype=torch.float16, device=DEV)
+    moeq4.moe_layer_decode(ctx, lay, x, T, y, idx, w, x_norm=xn if prenorm else None,
+                           flags=moeq4.MOE_PRENORM if prenorm else 0)
+    moeq4.moe_ctx_check(ctx)
+    close = assert_y_close_scaled if case == "extreme_raw" else assert_y_close
+    for t in sample:
+        xin = oracle.rmsnorm(x0[t], CFG.rms_eps) if prenorm else x0[t]
+        if prenorm:
+            np.testing.assert_array_equal(np_of(xn)[t], xin)
+        ref = oracle.moe_layer(CFG, Ln, xin)
+        assert idx[t].cpu().tolist() == ref["idx"].tolist(), f"{case} T={T} token {t}"
+        np.testing.assert_allclose(w[t].cpu().numpy(), ref["w"], rtol=2e-6, atol=1e-7)
+        close(y[t].cpu().numpy(), ref["y"], f"{case} T={T} token {t}")
+    ctx.close()
+
+
+def test_extreme_router_logits_exact(layer):
+    """The router alone on the fp16 extremes: logits equal the oracle's
+    exactly (the dot product is an exact integer; one rounding per step)."""
+    L, Ln, _ = layer
+    T = 4
+    x = synth.extreme_tokens(T, CFG.H, seed=91, device=DEV)
+    ctx = moeq4.Context(CFG, T)
+    idx = torch.empty((T, CFG.k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, CFG.k), device=DEV)
+    lg = torch.empty((T, CFG.E), dtype=torch.float64, device=DEV)
+    moeq4.moe_router_topk(ctx, L["router_w"], L["router_scale"], L["router_bias"], x, T, idx, w, lg)
+    torch.cuda.synchronize()
+    for t in range(T):
+        ref = oracle.router_logits(Ln["router_w"], Ln["router_scale"], Ln["router_bias"],
+                                   np_of(x)[t], CFG.E, CFG.H)
+        np.testing.assert_array_equal(lg[t].cpu().numpy(), ref)
+        assert idx[t].cpu().tolist() == oracle.topk(ref, CFG.k).tolist()
+    ctx.close()

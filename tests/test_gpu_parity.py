@@ -414,3 +414,27 @@ def test_argument_checks():
     with pytest.raises(moeq4.MoeError) as ei:
         moeq4.moe_layer_decode(ctx, st, x, 1, y)
     assert ei.value.code == moeq4.MOE_ERR_INVALID_ARG
+
+
+def test_smaller_context_keeps_larger_context_working():
+    """Kernel shared-memory limits belong to the process: creating a context
+    for a small shape after a large one must not shrink them under the large
+    context (router, grouped kernels and the fused kernel all take more
+    shared memory at the layer shape)."""
+    big = ctx_for(LAYER, 4)
+    small = ctx_for(TINY, 4)
+    L = make_layer(LAYER, seed=12, bias_std=1.5)
+    lay = moeq4.Layer.from_dict(L)
+    Ln = np_layer(L)
+    for T in (3, 1):
+        x = synth.tokens(T, LAYER.H, seed=13 + T, device=DEV)
+        y = torch.empty((T, LAYER.H), device=DEV)
+        idx = torch.empty((T, LAYER.k), dtype=torch.int32, device=DEV)
+        moeq4.moe_layer_decode(big, lay, x, T, y, idx)
+        moeq4.moe_ctx_check(big)
+        for t in range(T):
+            ref = _oracle_layer(LAYER, Ln, np_of(x)[t])
+            assert idx[t].cpu().tolist() == ref["idx"].tolist()
+            assert_y_close(y[t].cpu().numpy(), ref["y"], f"T={T} token {t}")
+    small.close()
+    big.close()
