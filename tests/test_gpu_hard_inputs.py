@@ -8,8 +8,11 @@ Cases (rows from the seeded generators in synth):
   other 63, fed raw and through the RMSNorm prologue;
 - Student-t (3 degrees of freedom) heavy tails, raw and through RMSNorm;
 - fp16 extremes (+-65504, smallest and largest subnormals, zeros) fed raw:
-  the router must stay bit-exact; the FFN output is then of size 1e5 and up,
-  where the absolute bound scales with max |y| (gpu_util).
+  the router must stay bit-exact.
+Fed raw, the outlier and extreme rows make |y| reach thousands and more;
+there the absolute bound scales with max |y| (gpu_util.assert_y_close_scaled)
+while rel L2 stays at 1e-3.  Through RMSNorm (the stack's own input path) and
+for the Student-t rows the plain bounds apply.
 
 Routing (indices) is compared bit for bit, weights within the router tests'
 tolerance, y within rel L2 <= 1e-3 and max abs <= 2e-3.
@@ -72,7 +75,11 @@ def test_hard_activations(layer, case, T, tau, sample):
     moeq4.moe_layer_decode(ctx, lay, x, T, y, idx, w, x_norm=xn if prenorm else None,
                            flags=moeq4.MOE_PRENORM if prenorm else 0)
     moeq4.moe_ctx_check(ctx)
-    close = assert_y_close_scaled if case == "extreme_raw" else assert_y_close
+    # raw rows with 1000x channels or fp16 extremes give |y| in the thousands and
+    # beyond: there the absolute bound scales with max |y| (fp32 itself cannot
+    # meet a fixed 2e-3 on such outputs; the CUDA-core path, which dequantises
+    # exactly and accumulates in plain fp32, shows the same absolute error)
+    close = assert_y_close_scaled if case in ("outlier_raw", "extreme_raw") else assert_y_close
     for t in sample:
         xin = oracle.rmsnorm(x0[t], CFG.rms_eps) if prenorm else x0[t]
         if prenorm:
