@@ -31,7 +31,7 @@ EXPORTS = ("moe_ctx_create", "moe_ctx_destroy", "moe_ctx_check", "moe_ctx_trace"
            "moe_last_error", "moe_blob_bytes",
            "moe_router_topk", "moe_expert_ffn_q4", "moe_combine", "moe_lfu_init",
            "moe_cache_lookup_lfu", "moe_layer_decode", "moe_stack_decode",
-           "moe_router_topk_noalloc", "moe_set_mma_min_tokens")
+           "moe_router_topk_noalloc", "moe_set_mma_min_tokens", "moe_set_wait_ns")
 
 
 class MoeError(RuntimeError):
@@ -69,7 +69,7 @@ class CMoeLfuTable(ctypes.Structure):
 
 LFU_TABLE_BYTES = ctypes.sizeof(CMoeLfuTable)
 PAIR_BYTES = 16   # MoeFfnPair: blob pointer, int32 inter, int32 token
-TRACE_WORDS = 160  # per CTA trace record of the fused layer kernel
+TRACE_WORDS = 160  # per CTA trace record of the persistent decode kernel
 
 _lib = None
 
@@ -91,6 +91,7 @@ def load() -> ctypes.CDLL:
         "moe_ctx_trace": ([P, i32, P, i32], i32),
         "moe_ctx_info": ([P, ctypes.c_char_p, i32], i32),
         "moe_set_mma_min_tokens": ([P, i32], i32),
+        "moe_set_wait_ns": ([P, ctypes.c_ulonglong], i32),
         "moe_last_error": ([], ctypes.c_char_p),
         "moe_blob_bytes": ([i32, i32], ctypes.c_size_t),
         "moe_router_topk": ([P, P, P, P, P, i32, P, P, P, P], i32),
@@ -185,10 +186,15 @@ def moe_set_mma_min_tokens(ctx, min_tokens: int):
     _check(load().moe_set_mma_min_tokens(ctx.handle, int(min_tokens)))
 
 
+def moe_set_wait_ns(ctx, ns: int):
+    """moe_set_wait_ns: bound of every device wait of the context (ns)."""
+    _check(load().moe_set_wait_ns(ctx.handle, int(ns)))
+
+
 def moe_ctx_trace(ctx, enable=-1, read=False):
-    """Switch phase tracing of the fused layer kernel (1 on, 0 off, -1 keep);
-    with read=True return the last launch's records as an int64 array
-    [n_ctas, 16] (see moeq4.h)."""
+    """Switch phase tracing of the persistent decode kernel (1 on, 0 off, -1
+    keep); with read=True return the records as a uint64 array [n_ctas, 160]
+    (layout in moeq4.h)."""
     import numpy as np
     n = 1024 * TRACE_WORDS
     buf = np.zeros(n, dtype=np.uint64) if read else None

@@ -438,3 +438,45 @@ def test_smaller_context_keeps_larger_context_working():
             assert_y_close(y[t].cpu().numpy(), ref["y"], f"T={T} token {t}")
     small.close()
     big.close()
+
+
+def test_bounded_wait_gives_up_and_context_recovers(monkeypatch):
+    """Failure detection without a GPU fault.  A streaming layer runs as three
+    launches (router; shared expert; routed experts with the down rows), and
+    the last waits for every gate/up item of the step, the shared launch's
+    included.  The host withholds the shared launch (MOEQ4_WITHHOLD_SHARED_AT),
+    so that wait cannot be met: with a 1 ms bound the kernel gives up,
+    records MOE_ERR_TIMEOUT and leaves.  moe_ctx_check reports it and resets
+    the counters; the next resident and streaming calls on the same context
+    match the oracle."""
+    cfg = TINY
+    Ls = _stack_layers(cfg, 1, seed=41)
+    hs, slots, tables = _streaming_setup(cfg, Ls)
+    monkeypatch.setenv("MOEQ4_WITHHOLD_SHARED_AT", "0")
+    ctx = ctx_for(cfg, 1)
+    moeq4.moe_set_wait_ns(ctx, 1_000_000)
+    with pytest.raises(moeq4.MoeError) as ei:
+        moeq4.moe_set_wait_ns(ctx, 10)
+    assert ei.value.code == moeq4.MOE_ERR_INVALID_ARG
+    moeq4.moe_lfu_init(ctx, tables[0], cfg.S)
+    L = Ls[0]
+    st = moeq4.Layer(L["router_w"], L["router_scale"], L["router_bias"], L["shared"], None, hs[0],
+                     slots[0], tables[0])
+    rs = moeq4.Layer.from_dict(L)
+    cs = torch.cuda.Stream()
+    x = synth.tokens(3, cfg.H, seed=42, device=DEV)
+    y = torch.empty((1, cfg.H), device=DEV)
+    idx = torch.empty((1, cfg.k), dtype=torch.int32, device=DEV)
+    moeq4.moe_layer_decode(ctx, st, x[0:1], 1, y, copy_stream=cs)
+    with pytest.raises(moeq4.MoeError) as ei:
+        moeq4.moe_ctx_check(ctx)
+    assert ei.value.code == moeq4.MOE_ERR_TIMEOUT
+    moeq4.moe_ctx_check(ctx)                          # cleared
+    Ln = np_layer(L)
+    for t, lay in ((1, rs), (2, st)):
+        moeq4.moe_layer_decode(ctx, lay, x[t:t + 1], 1, y, idx, copy_stream=cs)
+        moeq4.moe_ctx_check(ctx)
+        ref = _oracle_layer(cfg, Ln, np_of(x)[t])
+        assert idx[0].cpu().tolist() == ref["idx"].tolist()
+        assert_y_close(y[0].cpu().numpy(), ref["y"], f"after recovery, token {t}")
+    ctx.close()
