@@ -57,7 +57,12 @@ namespace moeq4 {
 
 constexpr int kDecWarps = 12;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kDecRouteWarp = kDecWarps - 1;    // router rows, routing
+constexpr int kDecRouteWarp = kDecWarps - 1;    // router rows, routing, down copies
+constexpr int kDecGWarps = 11;                  // warps on the gate/up tiles
+constexpr int kDecGThreads = kDecGWarps * 32;
+constexpr int kDecGChunks = kDecGWarps * 8;     // 32-column chunks per round of a tile
+constexpr int kDecSbVec = 2;                    // 16-byte words of a tile's scales/biases per thread
+constexpr int kDecRouterVec = 8;                // 16-byte words of a router row per lane (hidden <= 4096)
 constexpr int kDecMaxLayers = 64;               // layers per launch (kernel parameter table)
 constexpr int kDecRouterLimbs = 6;
 constexpr int kDecDownRows = 8;                 // output rows per down block
@@ -71,7 +76,7 @@ enum : int { kDecRouter = 1, kDecShared = 2, kDecRouted = 4, kDecFull = 7 };
 
 // trace slots of a step
 enum { kDtStart = 0, kDtInput = 1, kDtX = 2, kDtRouterRow = 3, kDtRouting = 4, kDtGDone = 5,
-       kDtHSync = 6, kDtHPacked = 7, kDtDownDone = 8, kDtClaimsShared = 9, kDtClaimsRouted = 10 };
+       kDtHSync = 6, kDtHPacked = 7, kDtDownDone = 8 };
 
 struct DecLayer {
     const int8_t* Wr;          // router int8 [E][H]
@@ -103,7 +108,7 @@ struct DecArgs {
     const uint8_t* routed_base;  // non-null: routed blobs at routed_base + sel_src[j] * stride
     unsigned long long* rsum;    // [2][E][2] tagged halves of the exact router sums
     unsigned long long* hbuf;    // [2][H/2] tagged fp16 pairs of the residual between steps
-    float* hall;                 // [Is + k I] intermediate h: shared, then routed by position
+    uint32_t* dlimb;             // [(Is + k I) / 32][24] packed intermediate h: shared, then routed
     DecSync* sync;
     int* status;
     unsigned long long* trace;   // optional
@@ -291,7 +296,7 @@ __device__ __forceinline__ unsigned long long dec_order_key(double d) {
 // warp maximum of the lane heads; the picks are exact unless an unpicked
 // expert shares the k-th pick's 24-bit key (then full exact rounds over the
 // fp64 keys) or two picks share a key (then an exact rank sort of the picks).
-__device__ __forceinline__ void dec_topk(const double (&v)[8], int E, int k, int renorm, int lane,
+__device__ __noinline__ void dec_topk(const double (&v)[8], int E, int k, int renorm, int lane,
                                          int& sel, float& w) {
     constexpr int kPer = 8;
     double sel_l = 0.0, m = 0.0;
@@ -397,17 +402,14 @@ struct DecShared {
     const uint8_t* blob[MOE_MAX_TOPK];   // routed blobs of the current step
     float rw[MOE_MAX_TOPK];              // routing weights
     int route_tag;                       // step + 1 once blob / rw hold the step's routing
-    int claim;                           // next gate/up item of this CTA (per step)
-    int gdone;                           // gate/up items of this CTA done (per step)
+    int issued_tag;                      // step + 1 once the gate/up warps issued their last tile
     int abort;                           // a wait of this CTA gave up
-    int nl;                              // router digits in use
     unsigned xmax_bits;                  // largest |x| of the step (router digits)
-    double r;                            // RMSNorm factor of the step
-    unsigned long long ss[kDecWarps * 2];   // exact sums of squares per warp
+    long long ss[kDecWarps * 3];         // exact sum of squares, three int64 parts per warp
 };
 
 struct DecSmemLayout {
-    size_t xs, hs, xl, xt, ht, dst, red, hnew, rsc, rbs, cs, total;
+    size_t xs, hs, xl, xt, ht, dst, sbt, red2, hb, red, hnew, rsc, rbs, cs, total;
     size_t blk_bytes, rblk;
     __host__ __device__ DecSmemLayout(int H, int E, int k, int I, int Is, int n_blocks) {
         rblk = (size_t)kDecDownRows * (I / 2 + I / 16);                    // one routed expert's rows
@@ -420,6 +422,9 @@ struct DecSmemLayout {
         xt = take((size_t)(H / 32) * kDecXWords * 4);
         ht = take((size_t)((Is + k * I) / 32) * kDecHWords * 4);
         dst = take((size_t)n_blocks * blk_bytes);
+        sbt = take((size_t)2 * 2 * H);                                    // tile scales/biases, two tiles
+        red2 = take((size_t)kDecGWarps * 32 * 4);
+        hb = take(64);
         red = take((size_t)(MOE_MAX_TOPK + 1) * kDecDownRows * 4);
         hnew = take((size_t)kDecDownRows * 2);
         rsc = take((size_t)E * 8);
@@ -432,7 +437,52 @@ struct DecSmemLayout {
 // Number of q in [0, n) with q = r (mod G), r in [0, G).
 __device__ __forceinline__ int dec_count(int n, int r, int G) { return n > r ? (n - 1 - r) / G + 1 : 0; }
 
+// Bounded wait until a shared-memory word equals `want`; lane 0 polls, the
+// warp learns the outcome.  Gives up on the CTA's or the kernel's abort.
+__device__ __forceinline__ bool dec_wait_smem_eq(const DecArgs& a, DecShared* cs, const int* p, int want,
+                                                 int lane) {
+    bool ok = true;
+    if (lane == 0 && *(volatile const int*)p != want) {
+        const unsigned long long t0 = dec_now();
+        for (unsigned q = 0; *(volatile const int*)p != want; q++) {
+            __nanosleep(64);
+            if ((q & 15) == 15 && (*(volatile int*)&cs->abort || dec_aborted(a.status) ||
+                                   dec_now() - t0 > a.wait_ns)) {
+                dec_fail(a.status);
+                ok = false;
+                break;
+            }
+        }
+    }
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    fence_acq_rel_cta();                      // every lane reads what the flag publishes
+    return ok;
+}
+
+// Named barrier among `n` threads that also ORs a predicate over them, so that
+// every participant leaves with the same answer.
+__device__ __forceinline__ bool dec_bar_or(int id, int n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"(pred ? 1u : 0u), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+// cp.async of `bytes` (a multiple of 16) from global to shared memory by one warp.
+__device__ __forceinline__ void dec_copy_warp(uint32_t dst, const uint8_t* src, int bytes, int lane) {
+    for (int u = lane; u < bytes / 16; u += 32) cp_async16(dst + 16 * u, src + 16 * u);
+}
+
 // ----------------------------------------------------------------- kernel --
+// Thread roles: warps 0..10 (352 threads) take the gate/up tiles, warp 11
+// the router rows, the routing and the copies of the down weights; all 12
+// take the down blocks.  A gate/up thread owns one 32-column chunk of x
+// (chunk 8 w + (lane & 7), and + 88 m for wider rows) and 8 of the tile's 32
+// rows (lane >> 3, + 4, + 8, ...).
 template <int MAXC>
 __global__ void __launch_bounds__(kDecThreads, 1) k_moe_decode(const __grid_constant__ DecArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -444,6 +494,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_moe_decode(const __grid_cons
     uint32_t* xt = reinterpret_cast<uint32_t*>(smem + lay.xt);
     uint32_t* ht = reinterpret_cast<uint32_t*>(smem + lay.ht);
     uint8_t* dst = smem + lay.dst;
+    uint8_t* sbt = smem + lay.sbt;
+    float* red2 = reinterpret_cast<float*>(smem + lay.red2);
+    uint32_t* hb = reinterpret_cast<uint32_t*>(smem + lay.hb);
     float* red = reinterpret_cast<float*>(smem + lay.red);
     __half* hnew = reinterpret_cast<__half*>(smem + lay.hnew);
     double* rsc = reinterpret_cast<double*>(smem + lay.rsc);
@@ -455,64 +508,134 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_moe_decode(const __grid_cons
     const int nch = H / 32;
     const bool m_router = (a.mode & kDecRouter) != 0, m_shared = (a.mode & kDecShared) != 0,
                m_routed = (a.mode & kDecRouted) != 0;
-    // this CTA's share of a step: router rows e = c (mod G); gate/up items
-    // dealt round-robin, shared indices first, then routed (slot j, index i)
-    // as f = j I + i after them; down blocks b = c (mod G)
+    // this CTA's share of a step: router rows e = c (mod G); gate/up tiles
+    // (16 intermediate indices of one expert) dealt round-robin, the shared
+    // expert's first, then the routed ones (slot j, tile q) as f = j I/16 + q;
+    // down blocks b = c (mod G)
     const int nR = m_router ? dec_count(E, c, G) : 0;
-    const int n_sh = m_shared ? Is : 0, n_rt = m_routed ? k * I : 0;
+    const int n_sh = m_shared ? Is / 16 : 0, n_rt = m_routed ? k * I / 16 : 0;
     const int nSG = dec_count(n_sh, c, G);
     const int rt0 = ((c - n_sh % G) % G + G) % G;          // first routed f with n_sh + f = c (mod G)
     const int nRG = dec_count(n_rt, rt0, G);
-    const int nG = nSG + nRG;
+    const int nGt = nSG + nRG;
     const int NB = H / kDecDownRows;
     const int nB = m_routed ? dec_count(NB, c, G) : 0;
-    const bool need_x = nR + nG > 0;
+    const bool need_x = nR + nGt > 0;
     const bool need_input = need_x || nB > 0;
     // the routing is computed where routed work needs it, and by CTA 0 of a
     // router launch for the caller's outputs
     const bool need_route = nRG > 0 || nB > 0 || (m_router && c == 0);
-    // gate/up items of a step over the grid, shared and routed: a launch with
-    // down blocks waits for all of them (in a split step the shared items come
-    // from the preceding shared launch, whose count the counter still holds)
+    // intermediate indices of a step over the grid, shared and routed: a
+    // launch with down blocks waits for all of them (in a split step the shared
+    // ones come from the preceding shared launch, whose count the counter holds)
     const unsigned long long ngu_step = (unsigned long long)(Is + k * I);
+    const int tpe = I / 16;                                 // gate/up tiles per routed expert
+    const BlobLayout Lr(H, I), Lsh(H, Is);
 
     const unsigned long long base = ld_rlx64(&a.sync->steps);
     const int S = a.n_layers * a.n_tokens;
-    if (tid == 0) { cs->abort = 0; cs->route_tag = 0; }
+    if (tid == 0) { cs->abort = 0; cs->route_tag = 0; cs->issued_tag = 0; }
     __syncthreads();
 
+#pragma unroll 1
     for (int s = 0; s < S; s++) {
         const int t = s / a.n_layers, l = s % a.n_layers;
         const DecLayer& Ly = a.layer[l];
         const unsigned tag = (unsigned)(base + s + 1);
         dec_trace(a, s, kDtStart);
-        // the router warp's first row: loaded now, while the input is awaited
-        uint4 wpre[2 * MAXC];
-        if (warp == kDecRouteWarp && nR > 0) {
-            const uint4* wrow = reinterpret_cast<const uint4*>(Ly.Wr + (size_t)c * H);
+
+        // ---- input-independent loads, issued while the input is awaited:
+        // the router warp's first row, router scales and biases, the shared
+        // expert's down rows of this CTA's blocks; the gate/up warps' first tile
+        // when it belongs to the shared expert
+        uint4 wpre[kDecRouterVec];
+        if (warp == kDecRouteWarp) {
+            if (nR > 0) {
+                const uint4* wrow = reinterpret_cast<const uint4*>(Ly.Wr + (size_t)c * H);
 #pragma unroll
-            for (int m = 0; m < 2 * MAXC; m++) {
-                const int j = lane + 32 * m;
-                wpre[m] = j < H / 16 ? ldg_stream128(wrow + j) : make_uint4(0, 0, 0, 0);
+                for (int m = 0; m < kDecRouterVec; m++) {
+                    const int j = lane + 32 * m;
+                    wpre[m] = j < H / 16 ? ldg_stream128(wrow + j) : make_uint4(0, 0, 0, 0);
+                }
+            }
+            if (need_route && m_router)
+                for (int e = lane; e < E; e += 32) {
+                    rsc[e] = (double)__half2float(Ly.rscale[e]);
+                    rbs[e] = Ly.rbias ? (double)Ly.rbias[e] : 0.0;
+                }
+#pragma unroll 1
+            for (int q = 0; q < nB; q++) {
+                const int row0 = (c + G * q) * kDecDownRows;
+                const uint8_t* tile = Ly.shared + Lsh.dn_base + (size_t)(row0 >> 4) * Lsh.dn_tile;
+                const int rin = row0 & 15;
+                const uint32_t d = smem_u32(dst + (size_t)q * lay.blk_bytes + (size_t)k * lay.rblk);
+                dec_copy_warp(d, tile + (size_t)rin * (Is / 2), kDecDownRows * Is / 2, lane);
+                dec_copy_warp(d + kDecDownRows * Is / 2, tile + (size_t)8 * Is + (size_t)rin * (Is / 32),
+                              kDecDownRows * Is / 32, lane);
+                dec_copy_warp(d + kDecDownRows * Is / 2 + kDecDownRows * Is / 32,
+                              tile + (size_t)8 * Is + Is / 2 + (size_t)rin * (Is / 32), kDecDownRows * Is / 32, lane);
             }
         }
+        const bool gw = warp < kDecGWarps && nGt > 0;
+        const int rg = lane >> 3;                           // row group of a gate/up thread
+        uint4 qc[MAXC][8];                                  // the current tile's codes of this thread
+        uint4 sbc[kDecSbVec];                               // and its share of the tile's scales/biases
+        float wc = 1.f;
+        int hpc = 0;
+        bool have_route = false;
+        // loads of tile `it` of this CTA's list (false: the routing never came)
+        auto issue = [&](int it, uint4 (&q)[MAXC][8], uint4 (&sb)[kDecSbVec], float& w, int& hp) -> bool {
+            const uint8_t* tb;
+            if (it < nSG) {
+                const int qt = c + G * it;
+                tb = Ly.shared + (size_t)qt * 18 * H;
+                w = 1.f;
+                hp = 16 * qt;
+            } else {
+                if (!have_route) {
+                    if (!dec_wait_smem_eq(a, cs, &cs->route_tag, s + 1, lane)) return false;
+                    have_route = true;
+                }
+                const int f = rt0 + G * (it - nSG);
+                const int j = f / tpe, qt = f - j * tpe;
+                tb = cs->blob[j] + (size_t)qt * 18 * H;
+                w = cs->rw[j];
+                hp = Is + j * I + 16 * qt;
+            }
+#pragma unroll
+            for (int m = 0; m < MAXC; m++) {
+                const int cc = 8 * warp + (lane & 7) + kDecGChunks * m;
+#pragma unroll
+                for (int n = 0; n < 8; n++)
+                    q[m][n] = cc < nch ? ldg_stream128(tb + (size_t)(rg + 4 * n) * (H / 2) + 16 * cc)
+                                       : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int v = 0; v < kDecSbVec; v++) {
+                const int u = tid + kDecGThreads * v;
+                sb[v] = u < H / 8 ? ldg_stream128(tb + (size_t)16 * H + 16 * u) : make_uint4(0, 0, 0, 0);
+            }
+            return true;
+        };
+        bool cur_loaded = false;
+        if (gw && nSG > 0) { issue(0, qc, sbc, wc, hpc); cur_loaded = true; }
 
         // ---- step input: the previous step's tagged residual, or the caller's row
         if (need_input) {
-            if (tid == 0) { cs->claim = 0; cs->gdone = 0; cs->xmax_bits = 0; }
+            if (tid == 0) cs->xmax_bits = 0;
             if (s > 0) {
                 // wait for every word of the previous step's output (sequential
                 // decode: also at token boundaries, where the data is the next row)
-                const unsigned long long* hb = a.hbuf + (size_t)((base + s - 1) & 1) * (H / 2);
+                const unsigned long long* hbp = a.hbuf + (size_t)((base + s - 1) & 1) * (H / 2);
                 const unsigned want = (unsigned)(base + s);
                 bool ok = true;
                 for (int i = tid; i < H / 2; i += kDecThreads) {
-                    unsigned long long wd = ld_rlx64(hb + i);
+                    unsigned long long wd = ld_rlx64(hbp + i);
                     if ((unsigned)(wd >> 32) != want) {
                         const unsigned long long t0 = dec_now();
                         for (unsigned it = 0; (unsigned)(wd >> 32) != want; it++) {
                             __nanosleep(32);
-                            wd = ld_rlx64(hb + i);
+                            wd = ld_rlx64(hbp + i);
                             if ((it & 15) == 15 && (dec_aborted(a.status) || dec_now() - t0 > a.wait_ns)) {
                                 dec_fail(a.status);
                                 ok = false;
@@ -529,101 +652,99 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_moe_decode(const __grid_cons
                 const uint4* src = reinterpret_cast<const uint4*>(a.hin + (size_t)t * H);
                 for (int i = tid; i < H / 8; i += kDecThreads) reinterpret_cast<uint4*>(hs)[i] = __ldcg(src + i);
             }
-            __syncthreads();
-            if (cs->abort) break;
+            // exact sum of squares: X = h 2^24 (|X| < 2^40) split as
+            // X = xh 2^20 + xl; X^2 = xh^2 2^40 + 2 xh xl 2^20 + xl^2, three
+            // int64 sums combined once in 128 bits
+            if (__syncthreads_or(*(volatile int*)&cs->abort)) break;
             dec_trace(a, s, kDtInput);
-
-            // ---- x (exact RMSNorm when prenorm)
+            double r = 1.0;
             if (a.prenorm) {
-                unsigned __int128 acc = 0;
+                long long s2 = 0, s1 = 0, s0 = 0;
                 for (int cc = tid; cc < H; cc += kDecThreads) {
                     const long long X = half_fixed24(hs[cc]);
-                    acc += (unsigned __int128)((__int128)X * (__int128)X);
+                    const int xh = (int)(X >> 20);
+                    const unsigned xl0 = (unsigned)(X & 0xFFFFF);
+                    s2 += (long long)xh * xh;
+                    s1 += (long long)xh * (long long)xl0;
+                    s0 += (long long)((unsigned long long)xl0 * xl0);
                 }
-                acc = warp_sum_u128(acc);
-                if (lane == 0) {
-                    cs->ss[2 * warp] = (unsigned long long)(acc >> 64);
-                    cs->ss[2 * warp + 1] = (unsigned long long)acc;
-                }
+                s2 = warp_sum(s2);
+                s1 = warp_sum(s1);
+                s0 = warp_sum(s0);
+                if (lane == 0) { cs->ss[3 * warp] = s2; cs->ss[3 * warp + 1] = s1; cs->ss[3 * warp + 2] = s0; }
                 __syncthreads();
-                if (tid == 0) {
-                    unsigned __int128 tot = 0;
-                    for (int w = 0; w < kDecWarps; w++)
-                        tot += ((unsigned __int128)cs->ss[2 * w] << 64) | cs->ss[2 * w + 1];
-                    const double sm = __dmul_rn(u128_to_double_rn(tot), 0x1p-48);
-                    const double ms = __ddiv_rn(sm, (double)H);
-                    cs->r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms, a.eps)));
-                }
-                __syncthreads();
-                const double r = cs->r;
-                for (int cc = tid; cc < H; cc += kDecThreads)
-                    xs[cc] = __double2half(__dmul_rn((double)__half2float(hs[cc]), r));
-            } else {
-                for (int i = tid; i < H / 8; i += kDecThreads)
-                    reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(hs)[i];
+                __int128 tot = 0;
+                for (int w = 0; w < kDecWarps; w++)
+                    tot += (__int128)cs->ss[3 * w] * ((__int128)1 << 40) +
+                           (__int128)cs->ss[3 * w + 1] * ((__int128)1 << 21) + (__int128)cs->ss[3 * w + 2];
+                const double sm = __dmul_rn(u128_to_double_rn((unsigned __int128)tot), 0x1p-48);
+                const double ms = __ddiv_rn(sm, (double)H);
+                r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms, a.eps)));
             }
-            __syncthreads();
-            if (c == 0 && s == 0 && a.x_norm_out)
-                for (int cc = tid; cc < H; cc += kDecThreads) a.x_norm_out[cc] = xs[cc];
-
-            // ---- router digits: x * 2^24 in balanced base-256 digits; NL
-            // digits cover this step's largest |x|
-            if (nR > 0) {
-                float mx = 0.f;
-                for (int cc = tid; cc < H; cc += kDecThreads) mx = fmaxf(mx, fabsf(__half2float(xs[cc])));
+            // x, the router's digits of x * 2^24 and the gate/up digit table:
+            // one thread per 8-column word (the 64-column group's largest |x|
+            // by shuffles over 8 consecutive threads)
+            float mx = 0.f;
+            for (int b0 = 0; b0 < H / 8; b0 += kDecThreads) {
+                const int wd = b0 + tid;
+                const bool valid = wd < H / 8;
+                float v[8];
+                uint4 xv = make_uint4(0, 0, 0, 0);
+                if (valid) {
+                    const uint4 hv = reinterpret_cast<const uint4*>(hs)[wd];
+                    if (a.prenorm) {
+                        const uint32_t hh[4] = {hv.x, hv.y, hv.z, hv.w};
+                        uint32_t xo[4];
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                if (lane == 0) atomicMax(&cs->xmax_bits, __float_as_uint(mx));
-                __syncthreads();
-                int NL = 1;
-                {
-                    const double xmax = (double)__uint_as_float(cs->xmax_bits) * 16777216.0;
-                    double cap = 127.0;
-                    while (NL < kDecRouterLimbs && xmax > cap) { NL++; cap = cap * 256.0 + 127.0; }
+                        for (int u = 0; u < 4; u++) {
+                            const __half2 p = *reinterpret_cast<const __half2*>(&hh[u]);
+                            const __half lo = __double2half(__dmul_rn((double)__low2float(p), r));
+                            const __half hi = __double2half(__dmul_rn((double)__high2float(p), r));
+                            xo[u] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+                        }
+                        xv = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+                    } else {
+                        xv = hv;
+                    }
+                    reinterpret_cast<uint4*>(xs)[wd] = xv;
                 }
-                if (tid == 0) cs->nl = NL;
-                for (int c4 = tid; c4 < H / 4; c4 += kDecThreads) {
-                    uint32_t packed[kDecRouterLimbs];
+                const uint32_t xq[4] = {xv.x, xv.y, xv.z, xv.w};
+                float m = 0.f, sx = 0.f;
 #pragma unroll
-                    for (int dg = 0; dg < kDecRouterLimbs; dg++) packed[dg] = 0;
+                for (int u = 0; u < 4; u++) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&xq[u]));
+                    v[2 * u] = f.x;
+                    v[2 * u + 1] = f.y;
+                    m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+                    sx += f.x + f.y;
+                }
+                mx = fmaxf(mx, m);
+                if (valid && nR > 0) {
+                    // balanced base-256 digits of x * 2^24 (exact integers)
+                    uint32_t pk[2][kDecRouterLimbs];
 #pragma unroll
-                    for (int q = 0; q < 4; q++) {
-                        long long X = __float2ll_rn(__half2float(xs[4 * c4 + q]) * 16777216.0f);   // exact
+                    for (int n = 0; n < 8; n++) {
+                        long long X = __float2ll_rn(v[n] * 16777216.0f);
 #pragma unroll
                         for (int dg = 0; dg < kDecRouterLimbs; dg++) {
                             const int digit = (int)((X + 128) & 255) - 128;
-                            packed[dg] |= (uint32_t)(digit & 255) << (8 * q);
+                            const uint32_t byte = (uint32_t)(digit & 255) << (8 * (n & 3));
+                            if (n & 3) pk[n >> 2][dg] |= byte; else pk[n >> 2][dg] = byte;
                             X = (X - digit) >> 8;
                         }
                     }
 #pragma unroll
-                    for (int dg = 0; dg < kDecRouterLimbs; dg++)
-                        if (dg < NL) reinterpret_cast<uint32_t*>(xl + dg * H)[c4] = packed[dg];
-                }
-            }
-            // ---- x digit table for the gate/up items: one thread per
-            // 8-column code word (the 64-column group's largest |x| by shuffles)
-            if (nG > 0) {
-                for (int b0 = 0; b0 < H / 8; b0 += kDecThreads) {
-                    const int wd = b0 + tid;
-                    const bool valid = wd < H / 8;
-                    float v[8];
-                    float m = 0.f, sx = 0.f;
-                    const uint4 q = valid ? reinterpret_cast<const uint4*>(xs)[wd] : make_uint4(0, 0, 0, 0);
-                    const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                    for (int u = 0; u < 4; u++) {
-                        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&qq[u]));
-                        v[2 * u] = f.x;
-                        v[2 * u + 1] = f.y;
-                        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
-                        sx += f.x + f.y;
+                    for (int dg = 0; dg < kDecRouterLimbs; dg++) {
+                        reinterpret_cast<uint32_t*>(xl + dg * H)[2 * wd] = pk[0][dg];
+                        reinterpret_cast<uint32_t*>(xl + dg * H)[2 * wd + 1] = pk[1][dg];
                     }
-                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-                    sx += __shfl_xor_sync(0xffffffffu, sx, 1);
-                    sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+                }
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+                sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+                sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+                if (valid && nGt > 0) {
                     const int Eg = dec_block_exp(m);
                     const float sc = dec_exp2(23 - Eg);
                     uint32_t d2e = 0, d2o = 0, b1e = 0, b1o = 0, b0e = 0, b0o = 0;
@@ -631,53 +752,65 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_moe_decode(const __grid_cons
                     for (int n = 0; n < 8; n++) {
                         int X = __float2int_rn(v[n] * sc);
                         X = max(-8388608, min(X, 8388607));
-                        const uint32_t b0 = (uint32_t)X & 0xffu, b1 = ((uint32_t)X >> 8) & 0xffu,
-                                       d2 = (uint32_t)(X >> 16) & 0xffu;
+                        const uint32_t c0 = (uint32_t)X & 0xffu, c1 = ((uint32_t)X >> 8) & 0xffu,
+                                       c2 = (uint32_t)(X >> 16) & 0xffu;
                         const int sh = 8 * (n >> 1);
-                        if (n & 1) { d2o |= d2 << sh; b1o |= b1 << sh; b0o |= b0 << sh; }
-                        else       { d2e |= d2 << sh; b1e |= b1 << sh; b0e |= b0 << sh; }
+                        if (n & 1) { d2o |= c2 << sh; b1o |= c1 << sh; b0o |= c0 << sh; }
+                        else       { d2e |= c2 << sh; b1e |= c1 << sh; b0e |= c0 << sh; }
                     }
-                    if (valid) {
-                        const int cch = wd >> 2, j = wd & 3;
-                        uint32_t* d = xt + (size_t)cch * kDecXWords;
-                        d[j] = d2e; d[4 + j] = d2o; d[8 + j] = b1e; d[12 + j] = b1o; d[16 + j] = b0e;
-                        d[20 + j] = b0o;
-                        if (j == 0) {
-                            d[24] = __float_as_uint(dec_exp2(Eg - 23));
-                            d[25] = __float_as_uint(sx);
-                        }
+                    const int cch = wd >> 2, j = wd & 3;
+                    uint32_t* d = xt + (size_t)cch * kDecXWords;
+                    d[j] = d2e; d[4 + j] = d2o; d[8 + j] = b1e; d[12 + j] = b1o; d[16 + j] = b0e;
+                    d[20 + j] = b0o;
+                    if (j == 0) {
+                        d[24] = __float_as_uint(dec_exp2(Eg - 23));
+                        d[25] = __float_as_uint(sx);
                     }
                 }
             }
+            if (nR > 0) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                if (lane == 0) atomicMax(&cs->xmax_bits, __float_as_uint(mx));
+            }
             __syncthreads();
+            if (c == 0 && s == 0 && a.x_norm_out)
+                for (int cc = tid; cc < H; cc += kDecThreads) a.x_norm_out[cc] = xs[cc];
             dec_trace(a, s, kDtX);
         }
 
-        // ---- router rows and the routing (one warp)
+        // ---- router rows, the routing, the routed down copies (router warp)
         if (warp == kDecRouteWarp) {
             const int slot = (int)((base + s) & 1);
             if (nR > 0) {
-                const int NL = cs->nl;
+                int NL = 1;
+                {
+                    const double xmax = (double)__uint_as_float(cs->xmax_bits) * 16777216.0;
+                    double cap = 127.0;
+                    while (NL < kDecRouterLimbs && xmax > cap) { NL++; cap = cap * 256.0 + 127.0; }
+                }
+#pragma unroll 1
                 for (int e = c; e < E; e += G) {
                     const uint4* wrow = reinterpret_cast<const uint4*>(Ly.Wr + (size_t)e * H);
                     int acc[kDecRouterLimbs];
 #pragma unroll
                     for (int dg = 0; dg < kDecRouterLimbs; dg++) acc[dg] = 0;
 #pragma unroll
-                    for (int m = 0; m < 2 * MAXC; m++) {
+                    for (int m = 0; m < kDecRouterVec; m++) {
                         const int j = lane + 32 * m;
-                        if (j >= H / 16) break;
-                        const uint4 w4 = e == c ? wpre[m] : ldg_stream128(wrow + j);
+                        if (j < H / 16) {
+                            const uint4 w4 = e == c ? wpre[m] : ldg_stream128(wrow + j);
 #pragma unroll
-                        for (int dg = 0; dg < kDecRouterLimbs; dg++) {
-                            if (dg < NL) {
-                                const uint4 l4 = lds128(smem_u32(xl + dg * H) + 16 * j);
-                                int sacc = acc[dg];
-                                sacc = __dp4a((int)w4.x, (int)l4.x, sacc);
-                                sacc = __dp4a((int)w4.y, (int)l4.y, sacc);
-                                sacc = __dp4a((int)w4.z, (int)l4.z, sacc);
-                                sacc = __dp4a((int)w4.w, (int)l4.w, sacc);
-                                acc[dg] = sacc;
+                            for (int dg = 0; dg < kDecRouterLimbs; dg++) {
+                                if (dg < NL) {
+                                    const uint4 l4 = lds128(smem_u32(xl + dg * H) + 16 * j);
+                                    int sacc = acc[dg];
+                                    sacc = __dp4a((int)w4.x, (int)l4.x, sacc);
+                                    sacc = __dp4a((int)w4.y, (int)l4.y, sacc);
+                                    sacc = __dp4a((int)w4.z, (int)l4.z, sacc);
+                                    sacc = __dp4a((int)w4.w, (int)l4.w, sacc);
+                                    acc[dg] = sacc;
+                                }
                             }
                         }
                     }
@@ -700,18 +833,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_moe_decode(const __grid_cons
                 float wgt = 0.f;
                 bool ok = true;
                 if (m_router) {
-                    // scales and biases of the router rows (weights: no wait)
-                    for (int e = lane; e < E; e += 32) {
-                        rsc[e] = (double)__half2float(Ly.rscale[e]);
-                        rbs[e] = Ly.rbias ? (double)Ly.rbias[e] : 0.0;
-                    }
                     // every expert's tagged sum halves of this step
                     const unsigned long long* rb = a.rsum + (size_t)slot * E * 2;
                     double v[8];
                     const unsigned long long t0 = dec_now();
-                    for (int i = 0; i < 8; i++) {
+#pragma unroll
+                    for (int i = 0; i < 8; i++) v[i] = 0.0;
+#pragma unroll 1
+                    for (int i = 0; i < 8 && ok; i++) {
                         const int e = lane + 32 * i;
-                        v[i] = 0.0;
                         if (e < E) {
                             unsigned long long w0 = ld_rlx64(rb + 2 * e), w1 = ld_rlx64(rb + 2 * e + 1);
                             for (unsigned it = 0; (unsigned)(w0 >> 32) != tag || (unsigned)(w1 >> 32) != tag; it++) {
@@ -724,13 +854,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_moe_decode(const __grid_cons
                                     break;
                                 }
                             }
-                            if (!ok) break;
-                            const long long Sv = (long long)(((w0 & 0xffffffffull) << 32) | (w1 & 0xffffffffull));
-                            double lg = __ll2double_rn(Sv);
-                            lg = __dmul_rn(lg, 0x1p-24);
-                            lg = __dmul_rn(lg, rsc[e]);
-                            if (Ly.rbias) lg = __dadd_rn(lg, rbs[e]);
-                            v[i] = lg;
+                            if (ok) {
+                                const long long Sv = (long long)(((w0 & 0xffffffffull) << 32) | (w1 & 0xffffffffull));
+                                double lg = __ll2double_rn(Sv);
+                                lg = __dmul_rn(lg, 0x1p-24);
+                                lg = __dmul_rn(lg, rsc[e]);
+                                if (Ly.rbias) lg = __dadd_rn(lg, rbs[e]);
+                                if (i == 0) v[0] = lg; else if (i == 1) v[1] = lg; else if (i == 2) v[2] = lg;
+                                else if (i == 3) v[3] = lg; else if (i == 4) v[4] = lg; else if (i == 5) v[5] = lg;
+                                else if (i == 6) v[6] = lg; else v[7] = lg;
+                            }
                         }
                     }
                     ok = __all_sync(0xffffffffu, ok);
@@ -759,17 +892,42 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_moe_decode(const __grid_cons
                         fence_acq_rel_cta();
                         *(volatile int*)&cs->route_tag = s + 1;
                     }
+                    __syncwarp();
                     dec_trace(a, s, kDtRouting);
+                    // the routed experts' down rows of this CTA's blocks, queued
+                    // behind the gate/up tiles (which the step needs first)
+                    if (nB > 0 && (nGt == 0 || dec_wait_smem_eq(a, cs, &cs->issued_tag, s + 1, lane))) {
+#pragma unroll 1
+                        for (int q = 0; q < nB; q++) {
+                            const int row0 = (c + G * q) * kDecDownRows;
+                            const int rin = row0 & 15;
+#pragma unroll 1
+                            for (int j = 0; j < k; j++) {
+                                const uint8_t* tile = cs->blob[j] + Lr.dn_base + (size_t)(row0 >> 4) * Lr.dn_tile;
+                                const uint32_t d = smem_u32(dst + (size_t)q * lay.blk_bytes + (size_t)j * lay.rblk);
+                                dec_copy_warp(d, tile + (size_t)rin * (I / 2), kDecDownRows * I / 2, lane);
+                                dec_copy_warp(d + kDecDownRows * I / 2, tile + (size_t)8 * I + (size_t)rin * (I / 32),
+                                              kDecDownRows * I / 32, lane);
+                                dec_copy_warp(d + kDecDownRows * I / 2 + kDecDownRows * I / 32,
+                                              tile + (size_t)8 * I + I / 2 + (size_t)rin * (I / 32),
+                                              kDecDownRows * I / 32, lane);
+                            }
+                        }
+                    }
                 }
             }
         }
 
-        // ---- gate/up items, claimed by the warps of the CTA (shared first)
-        if (nG > 0) {
+        // ---- gate/up tiles (gate/up warps): register double buffer over the
+        // CTA's tiles; per tile, 8 rows x 32 columns per thread, partial row
+        // sums reduced over the warp's 8 chunks and then over the 11 warps in
+        // a fixed order; warp 0 forms h = w GELU(gate) up for the 16 indices
+        // and publishes them packed (16-bit fixed point per 8 values)
+        if (gw) {
             XDigits X[MAXC];
 #pragma unroll
             for (int m = 0; m < MAXC; m++) {
-                const int cc = lane + 32 * m;
+                const int cc = 8 * warp + (lane & 7) + kDecGChunks * m;
                 const uint32_t src = smem_u32(xt + (size_t)(cc < nch ? cc : 0) * kDecXWords);
                 const uint4 t0 = lds128(src), t1 = lds128(src + 16), t2 = lds128(src + 32),
                             t3 = lds128(src + 48), t4 = lds128(src + 64), t5 = lds128(src + 80),
@@ -783,146 +941,122 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_moe_decode(const __grid_cons
                 X[m].fexp = __uint_as_float(t6.x);
                 X[m].sx = __uint_as_float(t6.y);
             }
-            bool have_route = false;
-            for (;;) {
-                int it = 0;
-                if (lane == 0) it = atomicAdd(&cs->claim, 1);
-                it = __shfl_sync(0xffffffffu, it, 0);
-                if (it >= nG) break;
-                const uint8_t* blob;
-                float wgt;
-                int Ie, hidx;
-                if (it < nSG) {
-                    const int i = c + G * it;
-                    blob = Ly.shared; wgt = 1.f; Ie = Is; hidx = i;
-                } else {
-                    const int f = rt0 + G * (it - nSG);
-                    const int j = f / I;
-                    if (!have_route) {
-                        bool ok = true;
-                        if (lane == 0) {
-                            const unsigned long long t0 = dec_now();
-                            for (unsigned q = 0; *(volatile int*)&cs->route_tag != s + 1; q++) {
-                                __nanosleep(64);
-                                if ((q & 15) == 15 && (*(volatile int*)&cs->abort || dec_aborted(a.status) ||
-                                                       dec_now() - t0 > a.wait_ns)) {
-                                    dec_fail(a.status);
-                                    ok = false;
-                                    break;
-                                }
-                            }
-                        }
-                        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { cs->abort = 1; break; }
-                        fence_acq_rel_cta();          // every lane reads the published routing
-                        have_route = true;
-                    }
-                    blob = cs->blob[j]; wgt = cs->rw[j]; Ie = I; hidx = Is + f;
-                    (void)Ie;
-                }
-                const int i = hidx < Is ? hidx : (hidx - Is) % I;
-                const uint8_t* tile = blob + (size_t)(i >> 4) * 18 * H;
-                const int r = i & 15;
-                const uint8_t* gq = tile + (size_t)r * (H / 2);
-                const uint8_t* uq = tile + (size_t)(16 + r) * (H / 2);
-                const uint8_t* gsp = tile + (size_t)16 * H + (size_t)r * (H / 32);
-                const uint8_t* usp = gsp + H / 2;
-                const uint8_t* gbp = tile + (size_t)17 * H + (size_t)r * (H / 32);
-                const uint8_t* ubp = gbp + H / 2;
-                uint4 qg[MAXC], qu[MAXC];
-                uint32_t sg[MAXC], su[MAXC], bg[MAXC], bu[MAXC];
-#pragma unroll
-                for (int m = 0; m < MAXC; m++) {
-                    const int cc = lane + 32 * m;
-                    if (cc < nch) {
-                        qg[m] = ldg_stream128(gq + 16 * cc);
-                        qu[m] = ldg_stream128(uq + 16 * cc);
-                        const int go = 2 * (cc >> 1);
-                        sg[m] = ldg_stream16(gsp + go);
-                        su[m] = ldg_stream16(usp + go);
-                        bg[m] = ldg_stream16(gbp + go);
-                        bu[m] = ldg_stream16(ubp + go);
-                    }
-                }
-                float g = 0.f, u = 0.f;
-#pragma unroll
-                for (int m = 0; m < MAXC; m++) {
-                    const int cc = lane + 32 * m;
-                    if (cc < nch) {
-                        const float dg = dec_dot_x(qg[m], X[m]);
-                        const float du = dec_dot_x(qu[m], X[m]);
-                        g = fmaf(dec_h2f(sg[m]) * X[m].fexp, dg, g);
-                        g = fmaf(dec_h2f(bg[m]), X[m].sx, g);
-                        u = fmaf(dec_h2f(su[m]) * X[m].fexp, du, u);
-                        u = fmaf(dec_h2f(bu[m]), X[m].sx, u);
-                    }
-                }
-                g = warp_sum(g);
-                u = warp_sum(u);
-                if (lane == 0) {
-                    a.hall[hidx] = gelu_f(g, a.gelu) * u * wgt;
+            bool ok = true;
+            if (!cur_loaded) ok = issue(0, qc, sbc, wc, hpc);
+#pragma unroll 1
+            for (int it = 0; it < nGt; it++) {
+                uint4 qn[MAXC][8], sbn[kDecSbVec];
+                float wn = 1.f;
+                int hpn = 0;
+                const bool more = it + 1 < nGt;
+                if (more && ok) ok = issue(it + 1, qn, sbn, wn, hpn);
+                if (warp == 0 && lane == 0 && (!more || !ok)) {
                     fence_acq_rel_cta();
-                    if (atomicAdd(&cs->gdone, 1) + 1 == nG) {
+                    *(volatile int*)&cs->issued_tag = s + 1;
+                }
+                if (!ok && lane == 0) cs->abort = 1;
+                // this tile's scales and biases into shared memory
+                uint8_t* sbs = sbt + (size_t)(it & 1) * 2 * H;
+#pragma unroll
+                for (int v = 0; v < kDecSbVec; v++) {
+                    const int u = tid + kDecGThreads * v;
+                    if (u < H / 8) reinterpret_cast<uint4*>(sbs)[u] = sbc[v];
+                }
+                if (dec_bar_or(1, kDecGThreads, !ok || *(volatile int*)&cs->abort)) break;
+                float acc[8];
+#pragma unroll
+                for (int n = 0; n < 8; n++) acc[n] = 0.f;
+                const uint32_t sbs_s = smem_u32(sbs);
+#pragma unroll
+                for (int m = 0; m < MAXC; m++) {
+                    const int cc = 8 * warp + (lane & 7) + kDecGChunks * m;
+                    if (cc < nch) {
+                        const uint32_t g2 = 2u * (uint32_t)(cc >> 1);
+#pragma unroll
+                        for (int n = 0; n < 8; n++) {
+                            const int R = rg + 4 * n;
+                            const float d = dec_dot_x(qc[m][n], X[m]);
+                            const float sv = dec_h2f(lds16(sbs_s + (uint32_t)(R * (H / 32)) + g2));
+                            const float bv = dec_h2f(lds16(sbs_s + (uint32_t)(H + R * (H / 32)) + g2));
+                            acc[n] = fmaf(sv * X[m].fexp, d, acc[n]);
+                            acc[n] = fmaf(bv, X[m].sx, acc[n]);
+                        }
+                    }
+                }
+                // reduce over the 8 lanes of a row group: lane l ends with row
+                // group (l >> 3)'s sum of row l & 7 (tile row (l >> 3) + 4 (l & 7))
+#pragma unroll
+                for (int nn = 8, bit = 4; nn > 1; nn >>= 1, bit >>= 1) {
+                    const bool upper = (lane & bit) != 0;
+#pragma unroll
+                    for (int i = 0; i < nn / 2; i++) {
+                        const float send = upper ? acc[i] : acc[i + nn / 2];
+                        const float keep = upper ? acc[i + nn / 2] : acc[i];
+                        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+                    }
+                }
+                red2[warp * 32 + rg + 4 * (lane & 7)] = acc[0];
+                named_bar(1, kDecGThreads);
+                if (warp == 0) {
+                    // row `lane` over the 11 warps, fixed order; lanes 0..15 gate, 16..31 up
+                    float tot = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kDecGWarps; w++) tot += red2[w * 32 + lane];
+                    const float up = __shfl_down_sync(0xffffffffu, tot, 16);
+                    const float h = lane < 16 ? gelu_f(tot, a.gelu) * up * wc : 0.f;
+                    // two 8-value words (lanes 0..7, 8..15): exponent, 16-bit fixed point
+                    float m = fabsf(h), sx = h;
+#pragma unroll
+                    for (int o = 1; o < 8; o <<= 1) {
+                        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                        sx += __shfl_xor_sync(0xffffffffu, sx, o);
+                    }
+                    const int Eg = dec_block_exp(m);
+                    int Xv = __float2int_rn(h * dec_exp2(15 - Eg));
+                    Xv = max(-32768, min(Xv, 32767));
+                    uint8_t* bytes = reinterpret_cast<uint8_t*>(hb);      // [2 words][eh oh el ol][4]
+                    if (lane < 16) {
+                        const int wdx = lane >> 3, n = lane & 7;
+                        const int kind = (n & 1) ? 4 : 0;
+                        bytes[32 * wdx + kind + (n >> 1)] = (uint8_t)((Xv >> 8) & 0xff);
+                        bytes[32 * wdx + 8 + kind + (n >> 1)] = (uint8_t)(Xv & 0xff);
+                    }
+                    __syncwarp();
+                    if (lane == 0 || lane == 8) {
+                        const int wdx = lane >> 3;
+                        const uint32_t* wv = hb + 8 * wdx;
+                        const int gidx = hpc / 8 + wdx;                    // 8-value group of h
+                        uint32_t* d = a.dlimb + (size_t)(gidx >> 2) * kDecHWords + (gidx & 3);
+                        d[0] = wv[0];
+                        d[4] = wv[1];
+                        d[8] = wv[2];
+                        d[12] = wv[3];
+                        d[16] = __float_as_uint(dec_exp2(Eg - 15));
+                        d[20] = __float_as_uint(sx);
+                    }
+                    __syncwarp();
+                    if (lane == 0 && !more) {
                         fence_acq_rel_gpu();
-                        red_release_add(&a.sync->gu_done, (unsigned long long)nG);
+                        red_release_add(&a.sync->gu_done, 16ull * (unsigned long long)nGt);
                         dec_trace(a, s, kDtGDone);
                     }
+                }
+                if (more) {
+#pragma unroll
+                    for (int m = 0; m < MAXC; m++)
+#pragma unroll
+                        for (int n = 0; n < 8; n++) qc[m][n] = qn[m][n];
+#pragma unroll
+                    for (int v = 0; v < kDecSbVec; v++) sbc[v] = sbn[v];
+                    wc = wn;
+                    hpc = hpn;
                 }
             }
         }
 
-        // ---- down blocks: copy the weights in as soon as the routing is known,
-        // then wait for every gate/up item of the step, pack h, compute, combine
+        // ---- down blocks: every gate/up item of the step, then h, compute, combine
         if (nB > 0) {
-            // routing of this step (every warp; it is there already unless this
-            // CTA had no routed gate/up items)
-            {
-                bool ok = true;
-                if (lane == 0 && *(volatile int*)&cs->route_tag != s + 1) {
-                    const unsigned long long t0 = dec_now();
-                    for (unsigned q = 0; *(volatile int*)&cs->route_tag != s + 1; q++) {
-                        __nanosleep(64);
-                        if ((q & 15) == 15 && (*(volatile int*)&cs->abort || dec_aborted(a.status) ||
-                                               dec_now() - t0 > a.wait_ns)) {
-                            dec_fail(a.status);
-                            ok = false;
-                            break;
-                        }
-                    }
-                }
-                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) cs->abort = 1;
-                fence_acq_rel_cta();                  // every lane reads the published routing
-            }
-            // copy regions: per block, k routed experts (codes, scales, biases
-            // of 8 rows) and the shared expert (same); warp w takes regions
-            // w, w + 12, ...
-            const int nreg = nB * 3 * (k + 1);
-            const BlobLayout Lr(H, I), Lsh(H, Is);
-            if (!cs->abort) {
-                for (int rg = warp; rg < nreg; rg += kDecWarps) {
-                    const int q = rg / (3 * (k + 1)), rr = rg % (3 * (k + 1));
-                    const int j = rr / 3, part = rr % 3;
-                    const int b = c + G * q;
-                    const int row0 = b * kDecDownRows;
-                    const bool shared_e = j == k;
-                    const int Ie = shared_e ? Is : I;
-                    const uint8_t* blob = shared_e ? Ly.shared : cs->blob[j];
-                    const BlobLayout& L = shared_e ? Lsh : Lr;
-                    const uint8_t* tile = blob + L.dn_base + (size_t)(row0 >> 4) * L.dn_tile;
-                    const int rin = row0 & 15;
-                    const uint8_t* src;
-                    int bytes;
-                    uint8_t* dd = dst + (size_t)q * lay.blk_bytes + (size_t)j * lay.rblk;
-                    if (part == 0) { src = tile + (size_t)rin * (Ie / 2); bytes = kDecDownRows * Ie / 2; }
-                    else if (part == 1) { src = tile + (size_t)8 * Ie + (size_t)rin * (Ie / 32); bytes = kDecDownRows * Ie / 32;
-                                          dd += (size_t)kDecDownRows * Ie / 2; }
-                    else { src = tile + (size_t)8 * Ie + Ie / 2 + (size_t)rin * (Ie / 32); bytes = kDecDownRows * Ie / 32;
-                           dd += (size_t)kDecDownRows * Ie / 2 + (size_t)kDecDownRows * Ie / 32; }
-                    const uint32_t d0 = smem_u32(dd);
-                    for (int u = lane; u < bytes / 16; u += 32) cp_async16(d0 + 16 * u, src + 16 * u);
-                }
-            }
-            // all gate/up items of the step (every CTA)
-            if (tid == 0 && !cs->abort) {
+            if (tid == 0 && !*(volatile int*)&cs->abort) {
                 const unsigned long long target = (unsigned long long)(s + 1) * ngu_step;
                 unsigned long long v;
                 asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(&a.sync->gu_done) : "memory");
@@ -941,42 +1075,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_moe_decode(const __grid_cons
                 }
                 dec_trace(a, s, kDtHSync);
             }
-            __syncthreads();
-            if (cs->abort) { cp_async_commit_wait_all(); break; }
-            // pack h: per 8 values one exponent, 16-bit fixed point in two
-            // int8 limbs (even / odd columns), the 8-value sum
+            if (__syncthreads_or(*(volatile int*)&cs->abort)) { cp_async_commit_wait_all(); break; }
+            // the packed h of the step (all experts) into shared memory
             {
-                const int nvals = Is + k * I;
-                for (int gi = tid; gi < nvals / 8; gi += kDecThreads) {
-                    const float4 p0 = __ldcg(reinterpret_cast<const float4*>(a.hall) + 2 * gi);
-                    const float4 p1 = __ldcg(reinterpret_cast<const float4*>(a.hall) + 2 * gi + 1);
-                    const float v[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-                    float m = 0.f, sx = 0.f;
-#pragma unroll
-                    for (int n = 0; n < 8; n++) { m = fmaxf(m, fabsf(v[n])); sx += v[n]; }
-                    const int Eg = dec_block_exp(m);
-                    const float sc = dec_exp2(15 - Eg);
-                    uint32_t eh = 0, oh = 0, el = 0, ol = 0;
-#pragma unroll
-                    for (int n = 0; n < 8; n++) {
-                        int Xv = __float2int_rn(v[n] * sc);
-                        Xv = max(-32768, min(Xv, 32767));
-                        const uint32_t lo = (uint32_t)Xv & 0xffu, hi = ((uint32_t)Xv >> 8) & 0xffu;
-                        const int sh = 8 * (n >> 1);
-                        if (n & 1) { oh |= hi << sh; ol |= lo << sh; }
-                        else       { eh |= hi << sh; el |= lo << sh; }
-                    }
-                    uint32_t* d = ht + (size_t)(gi >> 2) * kDecHWords + (gi & 3);
-                    d[0] = eh; d[4] = oh; d[8] = el; d[12] = ol;
-                    d[16] = __float_as_uint(dec_exp2(Eg - 15));
-                    d[20] = __float_as_uint(sx);
-                }
+                const int nw = (Is + k * I) / 32 * kDecHWords / 4;       // uint4 words
+                for (int i = tid; i < nw; i += kDecThreads)
+                    reinterpret_cast<uint4*>(ht)[i] = __ldcg(reinterpret_cast<const uint4*>(a.dlimb) + i);
             }
             cp_async_commit_wait_all();
             __syncthreads();
             dec_trace(a, s, kDtHPacked);
             const int nsw = kDecWarps - k;                  // warps on the shared rows
             const uint32_t ht_s = smem_u32(ht);
+#pragma unroll 1
             for (int q = 0; q < nB; q++) {
                 const int b = c + G * q;
                 const int row0 = b * kDecDownRows;
@@ -1011,6 +1122,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_moe_decode(const __grid_cons
                     const uint32_t cb = st + (uint32_t)(k * lay.rblk);
                     const uint32_t sb0 = cb + (uint32_t)(kDecDownRows * Is / 2);
                     const uint32_t bb0 = sb0 + (uint32_t)(kDecDownRows * Is / 32);
+#pragma unroll 1
                     for (int cc = lane; cc < Is / 32; cc += 32) {
                         const HLimbs16 L = dec_load_h(ht_s + (uint32_t)(cc * kDecHWords * 4));
                         const uint32_t go = 2u * (uint32_t)(cc >> 1);
@@ -1053,11 +1165,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_moe_decode(const __grid_cons
             }
             dec_trace(a, s, kDtDownDone);
         }
-        __syncthreads();
-        if (cs->abort) break;
+        if (__syncthreads_or(*(volatile int*)&cs->abort)) break;
     }
-    // leave: the launch's last CTA resets the gate/up counter and advances the
-    // context's step count (read by the next launch on this context)
+    // leave: the launch's last CTA advances the context's step count and, when
+    // the launch consumed the gate/up counter, resets it (read by the next
+    // launch on this context)
     cp_async_commit_wait_all();
     __syncthreads();
     if (tid == 0) {

@@ -87,7 +87,7 @@ struct moe_ctx {
     DecSync* dsync = nullptr;
     unsigned long long* rsum = nullptr;   // [2][E][2] tagged router sums
     unsigned long long* hbuf = nullptr;   // [2][H/2] tagged residual pairs
-    float* hall = nullptr;                // [Is + k I] intermediate h
+    uint32_t* dlimb = nullptr;            // [(Is + k I) / 32][24] packed intermediate h
     int* status = nullptr;                // device status word (bounded waits)
     int n_sms = 0;
     bool dec_ok = false;
@@ -249,7 +249,7 @@ static cudaError_t setup_grouped(moe_ctx* c) {
 }
 
 // Enables the persistent decode kernel for single-token steps when the shape
-// fits it: hidden <= 4096 (x digits of up to 4 chunks per lane), routed
+// fits it: hidden <= 4096 (x digits of up to 2 chunks per thread), routed
 // intermediate <= 1024 (one 32-value chunk per lane in the down blocks), at
 // most kDecMaxBlocks down blocks per CTA, its shared memory within the limit,
 // and one CTA of 384 threads per SM.
@@ -261,15 +261,16 @@ static cudaError_t setup_dec(moe_ctx* c) {
     int coop = 0;
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
     if (e != cudaSuccess) return e;
-    const int maxc = (g.hidden / 32 + 31) / 32;
+    const int maxc = (g.hidden / 32 + kDecGChunks - 1) / kDecGChunks;   // chunk rounds of a tile
     const int nblocks = (g.hidden / kDecDownRows + c->n_sms - 1) / (c->n_sms > 0 ? c->n_sms : 1);
     c->d_blocks = nblocks;
     c->d_smem = dec_smem_bytes(g.hidden, g.n_experts, g.top_k, g.inter, g.inter_shared, nblocks);
-    c->dec_ok = coop && c->n_sms > 0 && g.hidden <= 4096 && maxc >= 1 && maxc <= 4 &&
+    c->dec_ok = coop && c->n_sms > 0 && g.hidden <= 4096 && maxc >= 1 && maxc <= 2 &&
+                g.hidden / 8 <= kDecGThreads * kDecSbVec &&
                 g.inter <= 1024 && nblocks <= kDecMaxBlocks && c->d_smem <= (size_t)optin;
     if (!c->dec_ok) return cudaSuccess;
     typedef void (*KFn)(const DecArgs);
-    static const KFn table[4] = {k_moe_decode<1>, k_moe_decode<2>, k_moe_decode<3>, k_moe_decode<4>};
+    static const KFn table[2] = {k_moe_decode<1>, k_moe_decode<2>};
     c->d_kernel = table[maxc - 1];
     cudaFuncAttributes fa{};
     e = cudaFuncGetAttributes(&fa, c->d_kernel);
@@ -317,7 +318,7 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     size_t o_status = take(sizeof(int));
     size_t o_rsum = take(2 * E * 2 * sizeof(unsigned long long));
     size_t o_hbuf = take(2 * (H / 2) * sizeof(unsigned long long));
-    size_t o_hall = take((k * (size_t)cfg->inter + cfg->inter_shared) * sizeof(float));
+    size_t o_dlimb = take((k * (size_t)cfg->inter + cfg->inter_shared) / 32 * kDecHWords * 4);
     size_t o_eoff = take((E + 1) * sizeof(int));
     size_t o_plist = take(T * k * sizeof(int));
     size_t o_hpl = take(2 * P * (size_t)c->maxI * sizeof(__nv_bfloat16));   // h hi / lo planes
@@ -350,7 +351,7 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
         c->status = (int*)(c->ws + o_status);
         c->rsum = (unsigned long long*)(c->ws + o_rsum);
         c->hbuf = (unsigned long long*)(c->ws + o_hbuf);
-        c->hall = (float*)(c->ws + o_hall);
+        c->dlimb = (uint32_t*)(c->ws + o_dlimb);
         c->trace = (unsigned long long*)(c->ws + o_trace);
         size_t nm = T * k * 2 + 4;
         e = cudaHostAlloc((void**)&c->miss_host, nm * sizeof(int32_t), cudaHostAllocMapped);
@@ -453,7 +454,7 @@ static int launch_dec(moe_ctx* c, const MoeLayer* layers, int n_layers, int T, c
     a.routed_base = static_cast<const uint8_t*>(routed_base);
     a.rsum = c->rsum;
     a.hbuf = c->hbuf;
-    a.hall = c->hall;
+    a.dlimb = c->dlimb;
     a.sync = c->dsync;
     a.status = c->status;
     a.trace = c->tracing ? c->trace : nullptr;
