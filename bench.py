@@ -164,10 +164,9 @@ def build_stack(device, n_layers):
             for l in range(n_layers)]
 
 
-def kernel_launches_per_step(n_layers):
-    # one launch of the persistent decode kernel decodes every token of a step
-    # through every layer (up to 64 layers per launch)
-    return 1 if n_layers <= 64 else -(-n_layers // 64)
+def kernel_launches_per_token(n_layers):
+    # per token: load + store kernels and one fused kernel per layer
+    return 2 + n_layers
 
 
 def run_ours(args):
@@ -195,18 +194,9 @@ def run_ours(args):
     ctx = moeq4.Context(cfg, 1)
     stream = torch.cuda.current_stream()
 
-    kev = []          # per timed step: events around the decode launch alone
-
-    def step(timed=False):
+    def step():
         h.copy_(h0)
-        if timed:
-            ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            ka.record(stream)
-            moeq4.moe_stack_decode(ctx, objs, h, T, y_last)
-            kb.record(stream)
-            kev.append((ka, kb))
-        else:
-            moeq4.moe_stack_decode(ctx, objs, h, T, y_last)
+        moeq4.moe_stack_decode(ctx, objs, h, T, y_last)
 
     def barrier():
         torch.cuda.synchronize()
@@ -223,11 +213,10 @@ def run_ours(args):
     torch.cuda.profiler.start()          # a profiler started with capture off records this region
     e0.record(stream)
     for _ in range(args.steps):
-        step(timed=True)
+        step()
     e1.record(stream)
     barrier()
     torch.cuda.profiler.stop()
-    kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
     clk = clocks.stop()
     ms = e0.elapsed_time(e1) / args.steps
     ms_max = max_over_ranks(ms, world, dev)
@@ -254,7 +243,8 @@ def run_ours(args):
     e2e_value = job_tokens_per_s(world, T, max_over_ranks(ms_e2e, world, dev))
 
     moeq4.moe_ctx_check(ctx)
-    roof = roofline(max_over_ranks(kernel_ms, world, dev), L, T, cfg)
+    # ---- dominant kernel: the fused layer kernel of one token-layer
+    roof = roofline(ctx, layers, cfg, dev, stream)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -276,7 +266,7 @@ def run_ours(args):
                              "~1.1 GB touched per token)"},
             "e2e": {"value": round(e2e_value, 3), "unit": UNIT,
                     "h2d_bytes_per_step": T * cfg.H * 2, "d2h_bytes_per_step": T * cfg.H * 2},
-            "gpu_launches": kernel_launches_per_step(L) * (1 if L <= 64 else T) * args.steps,
+            "gpu_launches": kernel_launches_per_token(L) * T * args.steps,
             "roofline": roof,
             "clocks": clk,
         }
@@ -289,11 +279,15 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-# DRAM bytes (read + write) per token-layer of the persistent decode kernel,
-# from an ncu capture of the kernel built from the source with this SHA-256;
-# any other source reports null (the counters describe a different kernel).
-KERNEL_SRC = os.path.join(ROOT, "bit_quantized_expert_int8_b200", "csrc", "decode_fused.cuh")
-TRAFFIC_BY_SOURCE = {}
+# DRAM bytes (read + write) of one launch of the fused layer kernel, from an
+# ncu capture of the kernel built from the source with this SHA-256; any other
+# source reports null (the counters describe a different kernel).
+KERNEL_SRC = os.path.join(ROOT, "bit_quantized_expert_int8_b200", "csrc", "layer_fused.cuh")
+TRAFFIC_BY_SOURCE = {
+    # ncu --set full, one launch of the 30-layer bench layers (hidden 2816,
+    # top-8): dram__bytes_read.sum 37,284,864 + dram__bytes_write.sum 43,008
+    "ab523b1bf6c48f302f20a8d0fa33bdea867f6816a4e0a6fbc4a69b12422ad079": 37327872,
+}
 
 
 def kernel_traffic():
@@ -303,29 +297,51 @@ def kernel_traffic():
     return TRAFFIC_BY_SOURCE.get(digest), digest
 
 
-def algorithmic_bytes(cfg):
-    """Bytes one token-layer must read: the router (int8 rows and fp16
-    scales) and the blobs of the shared expert and the k routed experts."""
-    from bit_quantized_expert_int8_b200 import synth
-    return (cfg.k * synth.blob_bytes(cfg.H, cfg.I) + synth.blob_bytes(cfg.H, cfg.Is)
-            + cfg.E * cfg.H + 2 * cfg.E)
+def roofline(ctx, layers, cfg, dev, stream):
+    """Average duration of the dominant kernel, the fused single-token layer
+    kernel (router + shared and 8 routed expert FFNs + combine), over graph
+    replays of one launch per layer of the stack, so no weight is
+    L2-resident between its uses; algorithmic bytes = the router plus the 9
+    experts' blobs the token reads."""
+    import torch
 
-
-def roofline(ms_per_step, n_layers, n_tokens, cfg):
-    """The dominant kernel is the persistent decode kernel, and one step of
-    the stack workload is one launch of it (every token through every layer):
-    achieved = algorithmic bytes of the launch / its duration, the step time
-    measured with CUDA events around the launch on its stream."""
+    from bit_quantized_expert_int8_b200 import moeq4, synth
     hbm, kind = peaks()
-    algo = algorithmic_bytes(cfg) * n_layers * n_tokens
-    us_tl = ms_per_step * 1e3 / (n_layers * n_tokens)
-    achieved = algo / (ms_per_step * 1e-3) / 1e9
-    traffic = kernel_traffic()[0]
-    return {"bound": "hbm", "kernel": "k_moe_decode (persistent: every token and layer of a step)",
+    n = len(layers)
+    reps = 20
+    # a distinct token for every launch of the graph, so no launch can profit
+    # from the routing (or the weights) of an earlier replay
+    xs = synth.tokens(n * reps, cfg.H, SEED + 77, dev)
+    y = torch.empty((1, cfg.H), dtype=torch.float32, device=dev)
+    objs = [moeq4.Layer.from_dict(d) for d in layers]
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for i, o in enumerate(objs):                          # warm up
+            moeq4.moe_layer_decode(ctx, o, xs[i:i + 1], 1, y, stream=side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for r in range(reps):
+                for i, o in enumerate(objs):
+                    j = r * n + i
+                    moeq4.moe_layer_decode(ctx, o, xs[j:j + 1], 1, y, stream=side)
+        for _ in range(2):
+            g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(side)
+        g.replay()
+        e1.record(side)
+    torch.cuda.synchronize()
+    moeq4.moe_ctx_check(ctx)
+    us = e0.elapsed_time(e1) * 1000.0 / (reps * n)
+    algo = (cfg.k * synth.blob_bytes(cfg.H, cfg.I) + synth.blob_bytes(cfg.H, cfg.Is)
+            + cfg.E * cfg.H + 2 * cfg.E)
+    achieved = algo / (us * 1e-6) / 1e9
+    return {"bound": "hbm", "kernel": "k_moe_layer_fused (one token, one layer)",
             "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(achieved / hbm, 4), "peak_kind": f"{kind} (hbm_gbs)",
-            "algorithmic_bytes_per_launch": algo, "us_per_token_layer": round(us_tl, 3),
-            "traffic": None if traffic is None else traffic * n_layers * n_tokens}
+            "algorithmic_bytes_per_launch": algo, "us_per_launch": round(us, 3),
+            "traffic": kernel_traffic()[0]}
 
 
 def cpu_baseline(layers, cfg, seconds, h0=None, n_sample_layers=2):
@@ -556,7 +572,7 @@ def run_batched(args):
         # useful multiply-adds of the FFNs: gate, up and down of k routed and the shared expert
         flop = 2.0 * T * 3 * cfg.H * (cfg.k * cfg.I + cfg.Is)
         if T == 1:
-            path = "persistent decode kernel"
+            path = "fused single-token kernel"
         elif T >= 32:
             path = ("tcgen05 kernels (shared expert, buckets of >= 4 pairs) + CUDA-core grouped "
                     "kernels (smaller buckets)")

@@ -5,8 +5,8 @@
 // TurboFieldfare article, "L'affirmation des 2 Go ..."; daily.steinslab
 // article, "Trois optimisations cles" item 1).  One warp per output row,
 // 128-bit loads of packed codes, fp32 accumulation.  This form serves any
-// list of (expert, token) pairs; single-token decode steps use the persistent
-// kernel in decode_fused.cuh.
+// list of (expert, token) pairs; the single-token layer path uses the fused
+// kernel in layer_fused.cuh.
 #pragma once
 #include "common.cuh"
 

@@ -39,7 +39,7 @@
 #include <cuda_bf16.h>
 #include "common.cuh"
 #include "grouped.cuh"
-#include "waits.cuh"
+#include "layer_fused.cuh"
 #include "ptx.cuh"
 
 namespace moeq4 {
@@ -400,7 +400,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ C
                 const int brow = brow0 + z * kMmaTok;
                 for (int c = 0; c < nk; c++, g++) {
                     const uint32_t slot = g % R, use = g / R;
-                    if (!bounded_wait_bar(&empty_slot[slot], (use & 1u) ^ 1u, status)) { ok = false; break; }
+                    if (!fused_wait_bar(&empty_slot[slot], (use & 1u) ^ 1u, status)) { ok = false; break; }
                     const uint32_t sl = s_ring + slot * S::kSlot;
                     mbar_arrive_expect_tx(&full_slot[slot], (uint32_t)S::kSlot);
                     tma_load_4d(sl + S::kBBytes, &tm_codes, 32 * c, 0, (DOWN ? 8 : 4) * (int)blockIdx.x,
@@ -419,9 +419,9 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ C
             for (int z = blockIdx.z; ok && z * kMmaTok < n; z += gridDim.z) {
                 for (int c = 0; c < nk; c++, g++) {
                     const uint32_t slot = g % R, ab = g % kTcABufs, tb = g % kTcAccBufs;
-                    if (!bounded_wait_bar(&full_slot[slot], (g / R) & 1u, status) ||
-                        !bounded_wait_bar(&full_a[ab], (g / kTcABufs) & 1u, status) ||
-                        !bounded_wait_bar(&acc_empty[tb], ((g / kTcAccBufs) & 1u) ^ 1u, status)) {
+                    if (!fused_wait_bar(&full_slot[slot], (g / R) & 1u, status) ||
+                        !fused_wait_bar(&full_a[ab], (g / kTcABufs) & 1u, status) ||
+                        !fused_wait_bar(&acc_empty[tb], ((g / kTcAccBufs) & 1u) ^ 1u, status)) {
                         ok = false;
                         break;
                     }
@@ -457,8 +457,8 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ C
         for (int z = blockIdx.z; ok && z * kMmaTok < n; z += gridDim.z) {
             for (int c = 0; c < nk; c++, g++) {
                 const uint32_t slot = g % R, ab = g % kTcABufs;
-                if (!bounded_wait_bar(&full_slot[slot], (g / R) & 1u, status) ||
-                    !bounded_wait_bar(&empty_a[ab], ((g / kTcABufs) & 1u) ^ 1u, status)) {
+                if (!fused_wait_bar(&full_slot[slot], (g / R) & 1u, status) ||
+                    !fused_wait_bar(&empty_a[ab], ((g / kTcABufs) & 1u) ^ 1u, status)) {
                     ok = false;
                     break;
                 }
@@ -483,7 +483,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ C
         const int fj = warp & 3, ch = (warp - 10) >> 2;   // TMEM lane quarter, column half
         const int fm = 32 * fj + lane;                    // A row (TMEM lane)
         const uint32_t t_lane = tmem + ((uint32_t)(32 * fj) << 16) + 32u * ch;
-        if (!bounded_wait_bar(&sc_full, 0, status)) ok = false;
+        if (!fused_wait_bar(&sc_full, 0, status)) ok = false;
         uint32_t g = 0;
         for (int z = blockIdx.z; ok && z * kMmaTok < n; z += gridDim.z) {
             const int t0 = z * kMmaTok, nt = min(kMmaTok, n - t0);
@@ -502,7 +502,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ C
             for (int q = 0; q < 32; q++) acc[q] = 0.f;
             for (int c = 0; c < nk; c++, g++) {
                 const uint32_t tb = g % kTcAccBufs;
-                if (!bounded_wait_bar(&acc_full[tb], (g / kTcAccBufs) & 1u, status)) { ok = false; break; }
+                if (!fused_wait_bar(&acc_full[tb], (g / kTcAccBufs) & 1u, status)) { ok = false; break; }
                 tc_fence_after();
                 if (on) {
                     float P[32];

@@ -153,4 +153,28 @@ __global__ void k_build_pairs(const void* shared_blob, int Is, const uint8_t* ba
     }
 }
 
+__global__ void k_copy_half_row(const __half* __restrict__ src, __half* __restrict__ dst,
+                                const int* __restrict__ cursor, int H, int src_indexed) {
+    const int t = *cursor;
+    const __half* s = src + (src_indexed ? (size_t)t * H : 0);
+    __half* d = dst + (src_indexed ? 0 : (size_t)t * H);
+    for (int c = threadIdx.x; c < H; c += blockDim.x) d[c] = s[c];
+}
+
+__global__ void k_copy_rows(const __half* __restrict__ src, __half* __restrict__ dst, int n) {
+    for (int c = threadIdx.x; c < n; c += blockDim.x) dst[c] = src[c];
+}
+
+__global__ void k_store_token(const __half* __restrict__ h_cur, const float* __restrict__ y,
+                              __half* __restrict__ h_all, float* __restrict__ y_all,
+                              int* __restrict__ cursor, int H) {
+    const int t = *cursor;
+    for (int c = threadIdx.x; c < H; c += blockDim.x) {
+        h_all[(size_t)t * H + c] = h_cur[c];
+        if (y_all) y_all[(size_t)t * H + c] = y[c];
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) *cursor = t + 1;
+}
+
 }  // namespace moeq4

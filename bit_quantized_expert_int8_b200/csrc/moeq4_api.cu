@@ -16,7 +16,7 @@
 #include "ffn_tc.cuh"
 #include "ffn_simple.cuh"
 #include "grouped.cuh"
-#include "decode_fused.cuh"
+#include "layer_fused.cuh"
 #include "misc.cuh"
 #include "router.cuh"
 
@@ -55,6 +55,12 @@ static inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; 
 static inline bool aligned4(const void* p) { return ((uintptr_t)p & 3u) == 0; }
 
 // ------------------------------------------------------------ context --
+struct StackKey {
+    std::vector<MoeLayer> layers;
+    moe_half* h = nullptr;
+    float* y_last = nullptr;
+};
+
 struct moe_ctx {
     MoeConfig cfg{};
     int maxT = 0;
@@ -71,31 +77,35 @@ struct moe_ctx {
     float* y_pairs = nullptr;
     __half* x_norm = nullptr;
     int32_t* slot_of = nullptr;
+    int* cursor = nullptr;
+    __half* h_cur = nullptr;
+    float* y_cur = nullptr;
     // mapped pinned host memory for the streaming miss list
     int32_t* miss_host = nullptr;    // [maxT*k*2 + 4]; last words hold n_miss
     int32_t* miss_dev = nullptr;
     int32_t* n_miss_host = nullptr;
     int32_t* n_miss_dev = nullptr;
     cudaEvent_t ev_lookup = nullptr, ev_copy = nullptr;
+    cudaStream_t cap_stream = nullptr;
+    // stack graph
+    cudaGraphExec_t stack_exec = nullptr;
+    StackKey stack_key;
     // host-side fault injection (tests): fail the Nth blob copy before issue;
     // leave out the Nth shared-expert launch of a streaming layer
     long fail_copy_at = -1;
     long copies_seen = 0;
     long withhold_shared_at = -1;
     long shared_launches = 0;
-    // persistent decode kernel (single-token steps)
-    DecSync* dsync = nullptr;
-    unsigned long long* rsum = nullptr;   // [2][E][2] tagged router sums
-    unsigned long long* hbuf = nullptr;   // [2][H/2] tagged residual pairs
-    uint32_t* dlimb = nullptr;            // [(Is + k I) / 32][24] packed intermediate h
-    int* status = nullptr;                // device status word (bounded waits)
+    unsigned long long wait_ns = kWaitNs;  // bound of every device wait of the fused kernel
+    unsigned long long* shared_tag = nullptr;   // hand-off word of split streaming layers
+    unsigned long long stream_seq = 0;          // streaming layer calls so far
+    // fused single-token layer kernel
+    FusedSync* fsync = nullptr;        // [4 modes][2 parities]
+    int* status = nullptr;             // device status word (bounded waits)
+    __half* h_alt = nullptr;           // ping-pong residual buffer
+    int fparity[4] = {0, 0, 0, 0};
     int n_sms = 0;
-    bool dec_ok = false;
-    void (*d_kernel)(const DecArgs) = nullptr;
-    size_t d_smem = 0;
-    int d_blocks = 0;                  // down blocks per CTA and step at most
-    int d_regs = 0, d_max_threads = 0;
-    unsigned long long wait_ns = 2000000000ull;   // bound of every device wait
+    bool fused_ok = false;
     bool grouped_ok = false;           // multi-token steps grouped by expert
     bool mma_ok = false;               // tensor-core kernels usable for this shape
     int mma_min_tok = 0;               // bucket size from which they run (0: never)
@@ -105,8 +115,14 @@ struct moe_ctx {
     float* xg_sum = nullptr;           // [maxT * (k + 1)][H / 64] their group sums
     int* e_off = nullptr;              // [E + 1] pairs per expert (prefix)
     int* plist = nullptr;              // [maxT * k] pair indices grouped by expert
-    unsigned long long* trace = nullptr;   // [n_sms * 160] phase stamps
+    uint32_t* dlimb = nullptr;         // packed intermediate of the fused kernel
+    unsigned long long* ysh = nullptr; // tagged shared-expert down output [H]
+    int f_stages = 0, f_stage_bytes = 0;
+    int f_regs = 0, f_max_threads = 0;
+    unsigned long long* trace = nullptr;   // [n_sms * 16] phase stamps
     bool tracing = false;
+    size_t f_smem = 0;
+    void (*f_kernel)(const FusedArgs) = nullptr;
 };
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -158,8 +174,10 @@ extern "C" int moe_ctx_destroy(moe_ctx* c) {
     if (!c) return MOE_OK;
     cudaSetDevice(c->device);
     cudaDeviceSynchronize();
+    if (c->stack_exec) cudaGraphExecDestroy(c->stack_exec);
     if (c->ev_lookup) cudaEventDestroy(c->ev_lookup);
     if (c->ev_copy) cudaEventDestroy(c->ev_copy);
+    if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
     if (c->miss_host) cudaFreeHost(c->miss_host);
     if (c->ws) cudaFree(c->ws);
     delete c;
@@ -248,46 +266,49 @@ static cudaError_t setup_grouped(moe_ctx* c) {
     return cudaSuccess;
 }
 
-// Enables the persistent decode kernel for single-token steps when the shape
-// fits it: hidden <= 4096 (x digits of up to 2 chunks per thread), routed
-// intermediate <= 1024 (one 32-value chunk per lane in the down blocks), at
-// most kDecMaxBlocks down blocks per CTA, its shared memory within the limit,
-// and one CTA of 384 threads per SM.
-static cudaError_t setup_dec(moe_ctx* c) {
+// Chooses the fused kernel variant and its shared-memory ring for cfg.
+static cudaError_t setup_fused(moe_ctx* c) {
     const MoeConfig& g = c->cfg;
     int dev = c->device, optin = 0;
     cudaError_t e = cudaDeviceGetAttribute(&c->n_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    int coop = 0;
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
     if (e != cudaSuccess) return e;
-    const int maxc = (g.hidden / 32 + kDecGChunks - 1) / kDecGChunks;   // chunk rounds of a tile
-    const int nblocks = (g.hidden / kDecDownRows + c->n_sms - 1) / (c->n_sms > 0 ? c->n_sms : 1);
-    c->d_blocks = nblocks;
-    c->d_smem = dec_smem_bytes(g.hidden, g.n_experts, g.top_k, g.inter, g.inter_shared, nblocks);
-    c->dec_ok = coop && c->n_sms > 0 && g.hidden <= 4096 && maxc >= 1 && maxc <= 2 &&
-                g.hidden / 8 <= kDecGThreads * kDecSbVec &&
-                g.inter <= 1024 && nblocks <= kDecMaxBlocks && c->d_smem <= (size_t)optin;
-    if (!c->dec_ok) return cudaSuccess;
-    typedef void (*KFn)(const DecArgs);
-    static const KFn table[2] = {k_moe_decode<1>, k_moe_decode<2>};
-    c->d_kernel = table[maxc - 1];
+    const int nch = g.hidden / 32;
+    const int maxc = (nch + 31) / 32;
+    const int NCr = g.top_k * g.inter / 32, NCs = g.inter_shared / 32;
+    const int maxd = (NCr + 255) / 256;
+    // a stage holds one gate/up tile (18 H bytes), two shared down tiles
+    // (18 Is) or one down tile of each routed expert (9 I k)
+    size_t stage = (size_t)18 * g.hidden;
+    if ((size_t)18 * g.inter_shared > stage) stage = (size_t)18 * g.inter_shared;
+    if ((size_t)9 * g.inter * g.top_k > stage) stage = (size_t)9 * g.inter * g.top_k;
+    stage = (stage + 127) / 128 * 128;
+    int ns = 0;
+    for (int n = kFusedMaxStages; n >= 2 && ns == 0; n--)
+        if ((size_t)n * stage + fused_fixed_smem(g.hidden, NCr, NCs, n) <= (size_t)optin) ns = n;
+    c->fused_ok = g.hidden <= 4096 && maxc >= 1 && maxc <= 4 && maxd >= 1 && maxd <= 2 &&
+                  ns >= 2 && stage < (1u << 20) && c->n_sms > 0;
+    if (!c->fused_ok) return cudaSuccess;
+    typedef void (*KFn)(const FusedArgs);
+    static const KFn table[4][2] = {
+        {k_moe_layer_fused<1, 1>, k_moe_layer_fused<1, 2>},
+        {k_moe_layer_fused<2, 1>, k_moe_layer_fused<2, 2>},
+        {k_moe_layer_fused<3, 1>, k_moe_layer_fused<3, 2>},
+        {k_moe_layer_fused<4, 1>, k_moe_layer_fused<4, 2>}};
+    c->f_kernel = table[maxc - 1][maxd - 1];
     cudaFuncAttributes fa{};
-    e = cudaFuncGetAttributes(&fa, c->d_kernel);
+    e = cudaFuncGetAttributes(&fa, c->f_kernel);
     if (e != cudaSuccess) return e;
-    c->d_regs = fa.numRegs;
-    c->d_max_threads = fa.maxThreadsPerBlock;
-    if (fa.maxThreadsPerBlock < kDecThreads) {    // registers would not fit: use the direct kernels
-        c->dec_ok = false;
+    c->f_regs = fa.numRegs;
+    c->f_max_threads = fa.maxThreadsPerBlock;
+    if (fa.maxThreadsPerBlock < kFusedThreads) {    // registers would not fit: use the direct kernels
+        c->fused_ok = false;
         return cudaSuccess;
     }
-    e = raise_smem(c->d_kernel, c->d_smem);
-    if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, c->d_kernel, kDecThreads, c->d_smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) c->dec_ok = false;
-    return cudaSuccess;
+    c->f_stages = ns;
+    c->f_stage_bytes = (int)stage;
+    c->f_smem = (size_t)ns * stage + fused_fixed_smem(g.hidden, NCr, NCs, ns);
+    return raise_smem(c->f_kernel, (int)c->f_smem);
 }
 
 extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** out) {
@@ -314,11 +335,15 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     size_t o_y = take(P * H * sizeof(float));
     size_t o_xn = take(T * H * sizeof(__half));
     size_t o_slot = take(T * k * sizeof(int32_t));
-    size_t o_dsync = take(sizeof(DecSync));
+    size_t o_cur = take(sizeof(int));
+    size_t o_hcur = take(H * sizeof(__half));
+    size_t o_ycur = take(H * sizeof(float));
+    size_t o_fsync = take(8 * sizeof(FusedSync));
     size_t o_status = take(sizeof(int));
-    size_t o_rsum = take(2 * E * 2 * sizeof(unsigned long long));
-    size_t o_hbuf = take(2 * (H / 2) * sizeof(unsigned long long));
-    size_t o_dlimb = take((k * (size_t)cfg->inter + cfg->inter_shared) / 32 * kDecHWords * 4);
+    size_t o_stag = take(sizeof(unsigned long long));
+    size_t o_halt = take(H * sizeof(__half));
+    size_t o_dlimb = take((k * (size_t)cfg->inter + cfg->inter_shared) / 32 * kDLimbWords * 4);
+    size_t o_ysh = take(H * sizeof(unsigned long long));
     size_t o_eoff = take((E + 1) * sizeof(int));
     size_t o_plist = take(T * k * sizeof(int));
     size_t o_hpl = take(2 * P * (size_t)c->maxI * sizeof(__nv_bfloat16));   // h hi / lo planes
@@ -327,7 +352,7 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     size_t o_hsum = take(P * (size_t)(c->maxI / 64) * sizeof(float));        // h group sums
     int n_sms_dev = 0;
     cudaDeviceGetAttribute(&n_sms_dev, cudaDevAttrMultiProcessorCount, c->device);
-    size_t o_trace = take((size_t)(n_sms_dev > 0 ? n_sms_dev : 1) * 160 * sizeof(unsigned long long));
+    size_t o_trace = take((size_t)(n_sms_dev > 0 ? n_sms_dev : 1) * kTraceWords * sizeof(unsigned long long));
     int rc = MOE_OK;
     cudaError_t e = cudaMalloc(&c->ws, off);
     if (e == cudaSuccess) e = cudaMemset(c->ws, 0, off);
@@ -347,11 +372,15 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
         c->y_pairs = (float*)(c->ws + o_y);
         c->x_norm = (__half*)(c->ws + o_xn);
         c->slot_of = (int32_t*)(c->ws + o_slot);
-        c->dsync = (DecSync*)(c->ws + o_dsync);
+        c->cursor = (int*)(c->ws + o_cur);
+        c->h_cur = (__half*)(c->ws + o_hcur);
+        c->y_cur = (float*)(c->ws + o_ycur);
+        c->fsync = (FusedSync*)(c->ws + o_fsync);
         c->status = (int*)(c->ws + o_status);
-        c->rsum = (unsigned long long*)(c->ws + o_rsum);
-        c->hbuf = (unsigned long long*)(c->ws + o_hbuf);
+        c->shared_tag = (unsigned long long*)(c->ws + o_stag);
+        c->h_alt = (__half*)(c->ws + o_halt);
         c->dlimb = (uint32_t*)(c->ws + o_dlimb);
+        c->ysh = (unsigned long long*)(c->ws + o_ysh);
         c->trace = (unsigned long long*)(c->ws + o_trace);
         size_t nm = T * k * 2 + 4;
         e = cudaHostAlloc((void**)&c->miss_host, nm * sizeof(int32_t), cudaHostAllocMapped);
@@ -363,6 +392,7 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
         e = cudaEventCreateWithFlags(&c->ev_lookup, cudaEventDisableTiming);
     }
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_copy, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking);
     const int smem_router = (int)(H * sizeof(long long));
     if (e == cudaSuccess)
         e = raise_smem(k_router, smem_router);
@@ -371,7 +401,7 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     if (e == cudaSuccess)
         e = raise_smem(k_ffn_down_simple, (int)(c->maxI * sizeof(float)));
     if (e == cudaSuccess) e = setup_grouped(c);
-    if (e == cudaSuccess) e = setup_dec(c);
+    if (e == cudaSuccess) e = setup_fused(c);
     if (e != cudaSuccess) {
         rc = fail(MOE_ERR_CUDA, "moe_ctx_create: %s", cudaGetErrorString(e));
         moe_ctx_destroy(c);
@@ -420,62 +450,66 @@ static int launch_combine(moe_ctx* c, const float* y_routed, const float* y_shar
     return MOE_OK;
 }
 
-// A run of single-token decode steps on the persistent kernel: T tokens (rows
-// of hin) one after another, each through n_layers layers; or one part of a
-// split layer step (mode: router, shared expert, routed experts with the down
-// blocks).  Routed blobs are the layer's experts indexed by the routing, or
-// routed_base indexed by sel_src (the cache slots of a streaming layer).
-static int launch_dec(moe_ctx* c, const MoeLayer* layers, int n_layers, int T, const __half* hin,
-                      __half* hout, float* y, int32_t* idx_out, float* w_out, __half* x_norm_out,
-                      int prenorm, cudaStream_t s, int mode = kDecFull,
-                      const void* routed_base = nullptr, const int32_t* sel_src = nullptr) {
+// One token through one layer with the fused kernel.  `mode` selects the
+// work classes of this launch (kModeFull for a resident layer; streaming
+// splits it into router / shared / routed+down launches).  Routed blobs are
+// experts + sel[j] * stride with sel = the routing indices, or the cache
+// slots when `sel_slots` is given.
+static int launch_fused(moe_ctx* c, const MoeLayer* L, const __half* x_in, __half* h_out,
+                        __half* x_norm_out, float* y, int32_t* idx_out, float* w_out,
+                        int prenorm, cudaStream_t s, int mode = kModeFull,
+                        const void* experts = nullptr, const int32_t* sel_slots = nullptr,
+                        unsigned long long shared_seq = 0) {
     const MoeConfig& g = c->cfg;
-    if (n_layers < 1 || n_layers > kDecMaxLayers || T < 1)
-        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "decode launch: %d layers x %d tokens", n_layers, T);
-    DecArgs a{};
-    for (int l = 0; l < n_layers; l++) {
-        const MoeLayer& L = layers[l];
-        a.layer[l].Wr = L.router_w;
-        a.layer[l].rscale = reinterpret_cast<const __half*>(L.router_scale);
-        a.layer[l].rbias = L.router_bias;
-        a.layer[l].shared = static_cast<const uint8_t*>(L.shared_blob);
-        a.layer[l].experts = static_cast<const uint8_t*>(L.experts);
-    }
-    a.hin = hin;
-    a.hout = hout;
-    a.y = y;
-    a.idx_out = idx_out;
-    a.w_out = w_out;
+    const int mi = mode == kModeFull ? 0 : mode == kModeRouter ? 1 : mode == kModeShared ? 2 : 3;
+    FusedArgs a{};
+    a.Wr = L->router_w;
+    a.rscale = reinterpret_cast<const __half*>(L->router_scale);
+    a.rbias = L->router_bias;
+    a.shared = static_cast<const uint8_t*>(L->shared_blob);
+    a.experts = static_cast<const uint8_t*>(experts ? experts : L->experts);
+    a.stride = BlobLayout(g.hidden, g.inter).bytes;
+    a.sel_src = sel_slots ? sel_slots : c->idx;
+    a.x_in = x_in;
+    a.h_out = h_out;
     a.x_norm_out = x_norm_out;
+    a.y = y;
     a.idx_ws = c->idx;
     a.w_ws = c->w;
-    a.sel_src = sel_src ? sel_src : c->idx;
-    a.w_src = c->w;
-    a.routed_base = static_cast<const uint8_t*>(routed_base);
-    a.rsum = c->rsum;
-    a.hbuf = c->hbuf;
+    a.idx_out = idx_out;
+    a.w_out = w_out;
+    a.logits = c->logits;
     a.dlimb = c->dlimb;
-    a.sync = c->dsync;
+    a.ysh = c->ysh;
+    a.sync_id = 2 * mi + c->fparity[mi];
+    a.sync = c->fsync + a.sync_id;
+    c->fparity[mi] ^= 1;
     a.status = c->status;
     a.trace = c->tracing ? c->trace : nullptr;
     a.wait_ns = c->wait_ns;
-    a.stride = BlobLayout(g.hidden, g.inter).bytes;
+    a.shared_tag = shared_seq ? c->shared_tag : nullptr;
+    a.shared_seq = shared_seq;
     a.eps = g.rms_eps;
-    a.n_layers = n_layers; a.n_tokens = T; a.mode = mode; a.prenorm = prenorm;
     a.H = g.hidden; a.E = g.n_experts; a.k = g.top_k; a.I = g.inter; a.Is = g.inter_shared;
-    a.gelu = g.gelu; a.renorm = g.renorm;
-    a.max_blocks = c->d_blocks;
+    a.gelu = g.gelu; a.renorm = g.renorm; a.prenorm = prenorm;
+    a.n_stages = c->f_stages; a.stage_bytes = c->f_stage_bytes;
+    a.NR = (mode & kModeRouter) ? (g.n_experts + kRouterRows - 1) / kRouterRows : 0;
+    a.NSG = (mode & kModeShared) ? g.inter_shared / kGuRows : 0;
+    a.NRG = (mode & kModeRouted) ? g.top_k * (g.inter / kGuRows) : 0;
+    a.NSD = (mode & kModeDown) ? g.hidden / kSdRows : 0;
+    a.NRD = (mode & kModeDown) ? g.hidden / kRdRows : 0;
+    a.NTOT = a.NR + a.NSG + a.NSD + a.NRG + a.NRD;
     cudaLaunchConfig_t lc{};
     lc.gridDim = dim3(c->n_sms);
-    lc.blockDim = dim3(kDecThreads);
-    lc.dynamicSmemBytes = c->d_smem;
+    lc.blockDim = dim3(kFusedThreads);
+    lc.dynamicSmemBytes = c->f_smem;
     lc.stream = s;
     cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeCooperative;
-    at[0].val.cooperative = 1;
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = at;
     lc.numAttrs = 1;
-    CK(cudaLaunchKernelEx(&lc, c->d_kernel, a));
+    CK(cudaLaunchKernelEx(&lc, c->f_kernel, a));
     return MOE_OK;
 }
 
@@ -548,10 +582,16 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
                           int flags, cudaStream_t s) {
     const MoeConfig& g = c->cfg;
     const int k = g.top_k, H = g.hidden;
-    if (T == 1 && c->dec_ok) {
+    if (T == 1 && c->fused_ok) {
         const bool pre = (flags & MOE_PRENORM) != 0;
-        return launch_dec(c, L, 1, 1, x, pre ? x : nullptr, o->y, o->topk_idx, o->topk_w,
-                          reinterpret_cast<__half*>(o->x_norm), pre ? 1 : 0, s);
+        TRY(launch_fused(c, L, x, pre ? c->h_alt : nullptr,
+                         reinterpret_cast<__half*>(o->x_norm), o->y, o->topk_idx, o->topk_w,
+                         pre ? 1 : 0, s));
+        if (pre) {
+            k_copy_rows<<<1, 256, 0, s>>>(c->h_alt, x, H);
+            CKL();
+        }
+        return MOE_OK;
     }
     const __half* xin = x;
     __half* xn = o->x_norm ? reinterpret_cast<__half*>(o->x_norm) : c->x_norm;
@@ -686,35 +726,41 @@ static int issue_fills(moe_ctx* c, const MoeLayer* L, cudaStream_t s, cudaStream
     return MOE_OK;
 }
 
-// Streaming layer on the persistent kernel, split in three launches: router
-// (and the routing), then the cache lookup; the shared expert, which runs
-// while the host issues the fills; the routed experts from the cache slots
-// with the down blocks.  The three launches run the same item code as a
-// resident step, so the output is identical.
-static int layer_streaming_dec(moe_ctx* c, const MoeLayer* L, __half* x, const MoeLayerOut* o,
-                               int flags, cudaStream_t s, cudaStream_t cs) {
+// Streaming layer with the fused kernel: router launch, cache lookup, shared
+// branch launch overlapping the fills, then routed + down launch reading the
+// slots.  Same arithmetic as the resident fused launch, so identical output.
+static int layer_streaming_fused(moe_ctx* c, const MoeLayer* L, __half* x, const MoeLayerOut* o,
+                                 int flags, cudaStream_t s, cudaStream_t cs) {
     const MoeConfig& g = c->cfg;
     const int pre = (flags & MOE_PRENORM) ? 1 : 0;
     int32_t* slot_of = o->slot_of ? o->slot_of : c->slot_of;
-    TRY(launch_dec(c, L, 1, 1, x, nullptr, nullptr, o->topk_idx, o->topk_w,
-                   reinterpret_cast<__half*>(o->x_norm), pre, s, kDecRouter));
+    TRY(launch_fused(c, L, x, nullptr, reinterpret_cast<__half*>(o->x_norm), nullptr, o->topk_idx,
+                     o->topk_w, pre, s, kModeRouter));
     k_lfu_lookup<<<1, 32, 0, s>>>(L->lfu, c->idx, 1, g.top_k, slot_of, c->miss_dev, c->n_miss_dev);
     CKL();
     CK(cudaEventRecord(c->ev_lookup, s));
-    // host fault injection: the withheld shared launch leaves the routed
-    // launch's wait for the step's gate/up items unsatisfied (bounded wait)
+    // the shared launch hands its h to the routed launch through a tagged word
+    // (this call's sequence number); host fault injection can leave the shared
+    // launch out, so that the routed launch's bounded wait for it runs out
+    const unsigned long long seq = ++c->stream_seq;
     const bool withhold = c->withhold_shared_at >= 0 && c->shared_launches == c->withhold_shared_at;
     c->shared_launches++;
-    if (!withhold) TRY(launch_dec(c, L, 1, 1, x, nullptr, nullptr, nullptr, nullptr, nullptr, pre, s, kDecShared));
+    if (!withhold)
+        TRY(launch_fused(c, L, x, nullptr, nullptr, nullptr, nullptr, nullptr, pre, s, kModeShared,
+                         nullptr, nullptr, seq));
     TRY(issue_fills(c, L, s, cs));
-    TRY(launch_dec(c, L, 1, 1, x, pre ? x : nullptr, o->y, nullptr, nullptr, nullptr, pre, s,
-                   kDecRouted, L->slots, slot_of));
+    TRY(launch_fused(c, L, x, pre ? c->h_alt : nullptr, nullptr, o->y, nullptr, nullptr, pre, s,
+                     kModeRouted | kModeDown, L->slots, slot_of, seq));
+    if (pre) {
+        k_copy_rows<<<1, 256, 0, s>>>(c->h_alt, x, g.hidden);
+        CKL();
+    }
     return MOE_OK;
 }
 
 static int layer_streaming(moe_ctx* c, const MoeLayer* L, __half* x, const MoeLayerOut* o,
                            int flags, cudaStream_t s, cudaStream_t cs) {
-    if (c->dec_ok) return layer_streaming_dec(c, L, x, o, flags, s, cs);
+    if (c->fused_ok) return layer_streaming_fused(c, L, x, o, flags, s, cs);
     const MoeConfig& g = c->cfg;
     const int k = g.top_k, H = g.hidden, T = 1;
     const __half* xin = x;
@@ -788,23 +834,25 @@ extern "C" int moe_ctx_check(moe_ctx* c, moe_stream_t stream) {
     int st = 0;
     CK(cudaMemcpy(&st, c->status, sizeof(int), cudaMemcpyDeviceToHost));
     if (st == 0) return MOE_OK;
-    // a bounded wait gave up: clear the status and the decode kernel's
-    // counters so the context can be used again; step numbers restart, so the
-    // tagged words of earlier launches must not survive either
+    // a bounded wait gave up: clear the status and the launch counters so the
+    // context can be used again
     CK(cudaMemset(c->status, 0, sizeof(int)));
-    CK(cudaMemset(c->dsync, 0, sizeof(DecSync)));
-    CK(cudaMemset(c->rsum, 0, (size_t)2 * c->cfg.n_experts * 2 * sizeof(unsigned long long)));
-    CK(cudaMemset(c->hbuf, 0, (size_t)2 * (c->cfg.hidden / 2) * sizeof(unsigned long long)));
+    CK(cudaMemset(c->fsync, 0, 8 * sizeof(FusedSync)));
+    // epochs restart, so tagged words of earlier launches must not survive
+    CK(cudaMemset(c->ysh, 0, (size_t)c->cfg.hidden * sizeof(unsigned long long)));
+    CK(cudaMemset(c->shared_tag, 0, sizeof(unsigned long long)));
+    for (int m = 0; m < 4; m++) c->fparity[m] = 0;
     return fail(st, "a bounded device wait gave up (status %d); counters reset", st);
 }
 
 extern "C" int moe_ctx_info(moe_ctx* c, char* buf, int len) {
     if (!c || !buf || len < 1) return fail(MOE_ERR_INVALID_ARG, "moe_ctx_info: bad argument");
     int n = snprintf(buf, (size_t)len,
-                     "single-token path: %s; sms %d; threads %d; smem %zu B; registers %d; "
-                     "max threads %d; wait bound %llu ns",
-                     c->dec_ok ? "persistent decode kernel" : "direct kernels", c->n_sms, kDecThreads,
-                     c->d_smem, c->d_regs, c->d_max_threads, c->wait_ns);
+                     "single-token path: %s; sms %d; stages %d x %d B; smem %zu B; "
+                     "registers %d; max threads %d (needs %d); wait bound %llu ns",
+                     c->fused_ok ? "fused" : "direct kernels", c->n_sms, c->f_stages,
+                     c->f_stage_bytes, c->f_smem, c->f_regs, c->f_max_threads, kFusedThreads,
+                     c->wait_ns);
     return n < 0 ? fail(MOE_ERR_INVALID_ARG, "moe_ctx_info: format") : MOE_OK;
 }
 
@@ -819,7 +867,7 @@ extern "C" int moe_set_wait_ns(moe_ctx* c, unsigned long long ns) {
 extern "C" int moe_ctx_trace(moe_ctx* c, int enable, unsigned long long* host_out,
                              int max_words) {
     if (!c) return fail(MOE_ERR_INVALID_ARG, "moe_ctx_trace: NULL context");
-    const int words = c->n_sms * 160;
+    const int words = c->n_sms * kTraceWords;
     int n = 0;
     if (host_out) {
         CK(cudaDeviceSynchronize());
@@ -831,6 +879,11 @@ extern "C" int moe_ctx_trace(moe_ctx* c, int enable, unsigned long long* host_ou
         c->tracing = enable != 0;
     }
     return n;
+}
+
+static bool same_key(const StackKey& k, const MoeLayer* layers, int n, moe_half* h, float* y) {
+    if ((int)k.layers.size() != n || k.h != h || k.y_last != y) return false;
+    return memcmp(k.layers.data(), layers, sizeof(MoeLayer) * n) == 0;
 }
 
 extern "C" int moe_stack_decode(moe_ctx* c, const MoeLayer* layers, int n_layers, moe_half* h,
@@ -848,25 +901,40 @@ extern "C" int moe_stack_decode(moe_ctx* c, const MoeLayer* layers, int n_layers
             return fail(MOE_ERR_ALIGNMENT, "layer %d: pointers must be 16-byte aligned", l);
     }
     const int H = c->cfg.hidden;
-    __half* hh = reinterpret_cast<__half*>(h);
-    if (c->dec_ok && n_layers <= kDecMaxLayers)       // every token and layer in one launch
-        return launch_dec(c, layers, n_layers, T, hh, hh, y_last, nullptr, nullptr, nullptr, 1, stream);
-    for (int t = 0; t < T; t++) {
-        __half* row = hh + (size_t)t * H;
-        if (c->dec_ok) {                               // layers in runs of kDecMaxLayers
-            for (int l0 = 0; l0 < n_layers; l0 += kDecMaxLayers) {
-                const int nl = n_layers - l0 < kDecMaxLayers ? n_layers - l0 : kDecMaxLayers;
-                float* y = (l0 + nl == n_layers && y_last) ? y_last + (size_t)t * H : nullptr;
-                TRY(launch_dec(c, layers + l0, nl, 1, row, row, y, nullptr, nullptr, nullptr, 1, stream));
-            }
-        } else {
-            MoeLayerOut o{};
-            for (int l = 0; l < n_layers; l++) {
-                o.y = (l == n_layers - 1 && y_last) ? y_last + (size_t)t * H : c->y_pairs;
-                TRY(layer_resident(c, &layers[l], row, 1, &o, MOE_PRENORM, stream));
+    if (!c->stack_exec || !same_key(c->stack_key, layers, n_layers, h, y_last)) {
+        if (c->stack_exec) { cudaGraphExecDestroy(c->stack_exec); c->stack_exec = nullptr; }
+        cudaStream_t cs = c->cap_stream;
+        CK(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
+        int rc = MOE_OK;
+        k_copy_half_row<<<1, 256, 0, cs>>>(reinterpret_cast<__half*>(h), c->h_cur, c->cursor, H, 1);
+        MoeLayerOut o{};
+        o.y = c->y_cur;
+        __half* cur = c->h_cur;
+        for (int l = 0; l < n_layers && rc == MOE_OK; l++) {
+            if (c->fused_ok) {
+                __half* nxt = cur == c->h_cur ? c->h_alt : c->h_cur;
+                rc = launch_fused(c, &layers[l], cur, nxt, nullptr, c->y_cur, nullptr, nullptr, 1, cs);
+                cur = nxt;
+            } else {
+                rc = layer_resident(c, &layers[l], c->h_cur, 1, &o, MOE_PRENORM, cs);
             }
         }
+        if (rc == MOE_OK)
+            k_store_token<<<1, 256, 0, cs>>>(cur, c->y_cur, reinterpret_cast<__half*>(h), y_last,
+                                             c->cursor, H);
+        cudaGraph_t graph = nullptr;
+        cudaError_t e = cudaStreamEndCapture(cs, &graph);
+        if (rc != MOE_OK) { if (graph) cudaGraphDestroy(graph); return rc; }
+        if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "stack capture: %s", cudaGetErrorString(e));
+        e = cudaGraphInstantiate(&c->stack_exec, graph, 0);
+        cudaGraphDestroy(graph);
+        if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "stack instantiate: %s", cudaGetErrorString(e));
+        c->stack_key.layers.assign(layers, layers + n_layers);
+        c->stack_key.h = h;
+        c->stack_key.y_last = y_last;
     }
+    CK(cudaMemsetAsync(c->cursor, 0, sizeof(int), stream));
+    for (int t = 0; t < T; t++) CK(cudaGraphLaunch(c->stack_exec, stream));
     return MOE_OK;
 }
 

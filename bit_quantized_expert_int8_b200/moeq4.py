@@ -69,7 +69,7 @@ class CMoeLfuTable(ctypes.Structure):
 
 LFU_TABLE_BYTES = ctypes.sizeof(CMoeLfuTable)
 PAIR_BYTES = 16   # MoeFfnPair: blob pointer, int32 inter, int32 token
-TRACE_WORDS = 160  # per CTA trace record of the persistent decode kernel
+TRACE_WORDS = 160  # per CTA trace record of the fused layer kernel
 
 _lib = None
 
@@ -192,9 +192,9 @@ def moe_set_wait_ns(ctx, ns: int):
 
 
 def moe_ctx_trace(ctx, enable=-1, read=False):
-    """Switch phase tracing of the persistent decode kernel (1 on, 0 off, -1
-    keep); with read=True return the records as a uint64 array [n_ctas, 160]
-    (layout in moeq4.h)."""
+    """Switch phase tracing of the fused layer kernel (1 on, 0 off, -1 keep);
+    with read=True return the last launch's records as an int64 array
+    [n_ctas, 16] (see moeq4.h)."""
     import numpy as np
     n = 1024 * TRACE_WORDS
     buf = np.zeros(n, dtype=np.uint64) if read else None

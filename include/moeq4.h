@@ -104,15 +104,15 @@ int moe_ctx_destroy(moe_ctx *ctx);
 int moe_ctx_check(moe_ctx *ctx, moe_stream_t stream);
 
 /* One line describing the context: which kernels serve single-token layers
- * (the persistent decode kernel, or the direct kernels when the shape or the
- * device does not fit it), its shared memory, registers and wait bound.
- * Writes at most len bytes (NUL-terminated) into buf (host). */
+ * (the fused layer kernel, or the direct kernels when the shape or the device
+ * does not fit it), its shared-memory ring and register use.  Writes at most
+ * len bytes (NUL-terminated) into buf (host). */
 int moe_ctx_info(moe_ctx *ctx, char *buf, int len);
 
-/* Bound of every device wait of this context's kernels, in nanoseconds
- * (default 2e9).  When a wait runs out the kernel records MOE_ERR_TIMEOUT,
- * leaves, and moe_ctx_check reports it.  Host call, no device work.  Returns
- * MOE_ERR_INVALID_ARG outside 1e3 .. 6e10 ns. */
+/* Bound of every device wait of this context's fused layer kernel, in
+ * nanoseconds (default 2e9).  When a wait runs out the kernel records
+ * MOE_ERR_TIMEOUT and leaves; moe_ctx_check reports it.  Host call, no device
+ * work.  Returns MOE_ERR_INVALID_ARG outside 1e3 .. 6e10 ns. */
 int moe_set_wait_ns(moe_ctx *ctx, unsigned long long ns);
 
 /* Multi-token steps with all experts resident group the (token, expert)
@@ -132,15 +132,17 @@ int moe_set_wait_ns(moe_ctx *ctx, unsigned long long ns);
  * setting is then left unchanged). */
 int moe_set_mma_min_tokens(moe_ctx *ctx, int min_tokens);
 
-/* Tracing of the persistent decode kernel.  enable = 1 makes later launches
- * record, per CTA, 160 words; for each of the launch's first 4 steps, 12
- * globaltimer stamps (ns) at word 12 s + slot: 0 step start, 1 input ready,
- * 2 x ready, 3 router rows written, 4 routing known, 5 the CTA's last
- * gate/up item done, 6 every gate/up item of the step seen, 7 h packed,
- * 8 down blocks done; word 159 is the SM id.  Slots a CTA does not reach stay
- * 0.  enable = 0 stops recording, -1 leaves it as is.  When host_out is not
- * NULL the device is synchronised and up to max_words words are copied;
- * returns the number of words copied (>= 0) or an error. */
+/* Tracing of the single-token layer kernel.  enable = 1 makes later launches
+ * record, per CTA, 160 words: globaltimer stamps (ns) of kernel entry, end of
+ * the input prologue, first item, routing known, down phase ready, consumer
+ * end, producer end, top-k published; word 8 counts router / shared /
+ * routed / down items in 16-bit fields; word 9 is the SM id; words 10-18
+ * router item done, top-k start and steps, prologue steps; words 32.. hold,
+ * for the CTA's first 42 items, three stamps each (copies issued, data
+ * ready, item done): time in the low 56 bits, item type + 1 in bits 56-59.  enable = 0
+ * stops recording, -1 leaves it as is.  When host_out is not NULL the device
+ * is synchronised and up to max_words words of the last recorded launch are
+ * copied; returns the number of words copied (>= 0) or an error. */
 int moe_ctx_trace(moe_ctx *ctx, int enable, unsigned long long *host_out, int max_words);
 
 /* Message for the calling thread's most recent error ("" if none). */
@@ -314,9 +316,10 @@ int moe_cache_lookup_lfu(moe_ctx *ctx, MoeLfuTable *table,
  * missing blob on `copy`; `main` waits for the copies, runs the routed FFN
  * from the slots and combines.  The call returns after the copies are
  * issued (one host wait per call).  If issuing a copy fails the table is
- * marked invalid and MOE_ERR_CACHE_STATE is returned.  The three parts run
- * the same kernel code as a resident single-token layer, so streaming and
- * resident outputs are identical bit for bit.
+ * marked invalid and MOE_ERR_CACHE_STATE is returned.  The shared-expert part
+ * hands its intermediate to the routed part through a tagged word that the
+ * routed part waits for (bounded), so a missing shared part ends in
+ * MOE_ERR_TIMEOUT from moe_ctx_check rather than in wrong output.
  *
  * flags & MOE_PRENORM: `x` is the fp16 residual stream h; the layer input is
  * RMSNorm(h) (unit weight, eps = cfg.rms_eps, exact sum of squares, result
@@ -351,10 +354,9 @@ int moe_layer_decode(moe_ctx *ctx, const MoeLayer *layer, moe_half *x, int T,
  * Decodes T tokens one after another through n_layers resident layers
  * (each token: for every layer, x = RMSNorm(h), y = MoE(x), h <- fp16(h+y)),
  * the per-layer flow repeated over the layers and then per token ([RM]
- * "L'affirmation des 2 Go ...").  With up to 64 layers every token and layer
- * runs in one launch of the persistent decode kernel (a token starts once
- * the previous one has left the last layer); deeper stacks take one launch
- * per token and run of 64 layers.
+ * "L'affirmation des 2 Go ...").  The token loop runs as a captured CUDA
+ * graph replayed once per token; the first call for a given set of layers
+ * captures it.
  *   layers  host array [n_layers] of resident MoeLayer
  *   h       device fp16 [T][H], updated in place
  *   y_last  device fp32 [T][H] or NULL: MoE output of the last layer */
