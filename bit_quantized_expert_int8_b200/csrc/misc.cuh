@@ -70,11 +70,21 @@ k_combine(const float* __restrict__ y_routed, size_t routed_tok_stride,
 // miss in ascending order takes the lowest empty slot, else the slot unused by
 // this token with the lowest count, ties to the oldest insertion.  The table
 // is tiny and the walk is sequential: one thread.  grid 1, block 32.
+// An invalid table (an earlier fill failed) changes nothing: n_miss = -1,
+// slot_of is set to slot 0 (a valid index, so later kernels stay in bounds)
+// and, when status is given, MOE_ERR_CACHE_STATE is recorded there.
 __global__ void k_lfu_lookup(MoeLfuTable* __restrict__ tb, const int32_t* __restrict__ idx,
                              int T, int k, int32_t* __restrict__ slot_of,
-                             int32_t* __restrict__ miss_list, int32_t* __restrict__ n_miss) {
+                             int32_t* __restrict__ miss_list, int32_t* __restrict__ n_miss,
+                             int* __restrict__ status = nullptr) {
     if (threadIdx.x != 0) return;
-    if (!tb->valid) { *n_miss = -1; return; }
+    if (!tb->valid) {
+        for (int i = 0; i < T * k; i++) slot_of[i] = 0;
+        if (status) atomicCAS(status, 0, MOE_ERR_CACHE_STATE);
+        __threadfence_system();
+        *n_miss = -1;
+        return;
+    }
     const int S = tb->n_slots;
     int nm = 0;
     for (int t = 0; t < T; t++) {
@@ -127,6 +137,45 @@ __global__ void k_lfu_lookup(MoeLfuTable* __restrict__ tb, const int32_t* __rest
     }
     __threadfence_system();
     *n_miss = nm;
+}
+
+// Device-initiated cache fill: the blobs of the miss list, copied from pinned
+// host memory (read over the bus by plain 16-byte loads) into their cache
+// slots, with no host involvement ("Gemma 4 26B : Comment faire tourner un LLM
+// en 2 Go de RAM", section 04 "Le pipeline de traitement": only the missing
+// experts are loaded).  grid (parts, max misses), block 256: blockIdx.y is the
+// miss, blockIdx.x a part of its blob; nothing to do for misses beyond n_miss
+// (or when n_miss < 0).
+constexpr int kFillParts = 16;
+constexpr int kFillThreads = 256;
+
+__global__ void __launch_bounds__(kFillThreads)
+k_fill_from_host(const uint8_t* __restrict__ store, uint8_t* __restrict__ slots, size_t stride,
+                 const int32_t* __restrict__ miss_list, const int32_t* __restrict__ n_miss, int E, int S) {
+    const int j = blockIdx.y;
+    if (j >= *n_miss) return;
+    const int e = miss_list[2 * j], s = miss_list[2 * j + 1];
+    if (e < 0 || e >= E || s < 0 || s >= S) return;
+    const uint4* src = reinterpret_cast<const uint4*>(store + (size_t)e * stride);
+    uint4* dst = reinterpret_cast<uint4*>(slots + (size_t)s * stride);
+    const size_t n16 = stride / 16;
+    const size_t per = (n16 + gridDim.x - 1) / gridDim.x;
+    const size_t b0 = (size_t)blockIdx.x * per;
+    const size_t b1 = b0 + per < n16 ? b0 + per : n16;
+    constexpr int U = 4;                          // 16-byte loads in flight per thread
+    for (size_t i = b0 + threadIdx.x; i < b1; i += (size_t)kFillThreads * U) {
+        uint4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const size_t q = i + (size_t)u * kFillThreads;
+            v[u] = q < b1 ? __ldg(src + q) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const size_t q = i + (size_t)u * kFillThreads;
+            if (q < b1) dst[q] = v[u];
+        }
+    }
 }
 
 __global__ void k_lfu_init(MoeLfuTable* tb, int S) {

@@ -83,6 +83,8 @@ struct moe_ctx {
     // mapped pinned host memory for the streaming miss list
     int32_t* miss_host = nullptr;    // [maxT*k*2 + 4]; last words hold n_miss
     int32_t* miss_dev = nullptr;
+    int32_t* miss_list_d = nullptr;  // [maxT*k*2] miss list in device memory (device-initiated fill)
+    int32_t* n_miss_d = nullptr;
     int32_t* n_miss_host = nullptr;
     int32_t* n_miss_dev = nullptr;
     cudaEvent_t ev_lookup = nullptr, ev_copy = nullptr;
@@ -340,6 +342,7 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     size_t o_ycur = take(H * sizeof(float));
     size_t o_fsync = take(8 * sizeof(FusedSync));
     size_t o_status = take(sizeof(int));
+    size_t o_missd = take((T * k * 2 + 4) * sizeof(int32_t));
     size_t o_stag = take(sizeof(unsigned long long));
     size_t o_halt = take(H * sizeof(__half));
     size_t o_dlimb = take((k * (size_t)cfg->inter + cfg->inter_shared) / 32 * kDLimbWords * 4);
@@ -377,6 +380,8 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
         c->y_cur = (float*)(c->ws + o_ycur);
         c->fsync = (FusedSync*)(c->ws + o_fsync);
         c->status = (int*)(c->ws + o_status);
+        c->miss_list_d = (int32_t*)(c->ws + o_missd);
+        c->n_miss_d = c->miss_list_d + T * k * 2;
         c->shared_tag = (unsigned long long*)(c->ws + o_stag);
         c->h_alt = (__half*)(c->ws + o_halt);
         c->dlimb = (uint32_t*)(c->ws + o_dlimb);
@@ -729,14 +734,33 @@ static int issue_fills(moe_ctx* c, const MoeLayer* L, cudaStream_t s, cudaStream
 // Streaming layer with the fused kernel: router launch, cache lookup, shared
 // branch launch overlapping the fills, then routed + down launch reading the
 // slots.  Same arithmetic as the resident fused launch, so identical output.
+// The fills are either issued by the host (one cudaMemcpyAsync per missing
+// blob, after one host wait for the miss list) or, with MOE_DEVICE_FILL, by a
+// gather kernel on the copy stream that reads the miss list in device memory
+// and pulls the blobs from pinned host memory: no host wait at all.
 static int layer_streaming_fused(moe_ctx* c, const MoeLayer* L, __half* x, const MoeLayerOut* o,
                                  int flags, cudaStream_t s, cudaStream_t cs) {
     const MoeConfig& g = c->cfg;
     const int pre = (flags & MOE_PRENORM) ? 1 : 0;
+    const bool dev_fill = (flags & MOE_DEVICE_FILL) != 0;
     int32_t* slot_of = o->slot_of ? o->slot_of : c->slot_of;
+    const void* dstore = nullptr;
+    if (dev_fill) {
+        void* p = nullptr;
+        if (cudaHostGetDevicePointer(&p, const_cast<void*>(L->host_store), 0) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return fail(MOE_ERR_INVALID_ARG, "MOE_DEVICE_FILL needs host_store in pinned host memory "
+                                             "that the device can address");
+        }
+        dstore = p;
+    }
     TRY(launch_fused(c, L, x, nullptr, reinterpret_cast<__half*>(o->x_norm), nullptr, o->topk_idx,
                      o->topk_w, pre, s, kModeRouter));
-    k_lfu_lookup<<<1, 32, 0, s>>>(L->lfu, c->idx, 1, g.top_k, slot_of, c->miss_dev, c->n_miss_dev);
+    if (dev_fill)
+        k_lfu_lookup<<<1, 32, 0, s>>>(L->lfu, c->idx, 1, g.top_k, slot_of, c->miss_list_d, c->n_miss_d,
+                                      c->status);
+    else
+        k_lfu_lookup<<<1, 32, 0, s>>>(L->lfu, c->idx, 1, g.top_k, slot_of, c->miss_dev, c->n_miss_dev);
     CKL();
     CK(cudaEventRecord(c->ev_lookup, s));
     // the shared launch hands its h to the routed launch through a tagged word
@@ -748,7 +772,18 @@ static int layer_streaming_fused(moe_ctx* c, const MoeLayer* L, __half* x, const
     if (!withhold)
         TRY(launch_fused(c, L, x, nullptr, nullptr, nullptr, nullptr, nullptr, pre, s, kModeShared,
                          nullptr, nullptr, seq));
-    TRY(issue_fills(c, L, s, cs));
+    if (dev_fill) {
+        const size_t stride = BlobLayout(g.hidden, g.inter).bytes;
+        CK(cudaStreamWaitEvent(cs, c->ev_lookup, 0));
+        k_fill_from_host<<<dim3(kFillParts, g.top_k), kFillThreads, 0, cs>>>(
+            static_cast<const uint8_t*>(dstore), static_cast<uint8_t*>(L->slots), stride, c->miss_list_d,
+            c->n_miss_d, g.n_experts, MOE_MAX_SLOTS);
+        CKL();
+        CK(cudaEventRecord(c->ev_copy, cs));
+        CK(cudaStreamWaitEvent(s, c->ev_copy, 0));
+    } else {
+        TRY(issue_fills(c, L, s, cs));
+    }
     TRY(launch_fused(c, L, x, pre ? c->h_alt : nullptr, nullptr, o->y, nullptr, nullptr, pre, s,
                      kModeRouted | kModeDown, L->slots, slot_of, seq));
     if (pre) {
@@ -796,7 +831,7 @@ extern "C" int moe_layer_decode(moe_ctx* c, const MoeLayer* L, moe_half* x, int 
                                 const MoeLayerOut* o, int flags, moe_stream_t main,
                                 moe_stream_t copy) {
     if (!c || !L || !x || !o || !o->y) return fail(MOE_ERR_INVALID_ARG, "moe_layer_decode: NULL argument");
-    if (flags & ~MOE_PRENORM) return fail(MOE_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+    if (flags & ~(MOE_PRENORM | MOE_DEVICE_FILL)) return fail(MOE_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
     if (T < 1 || T > c->maxT) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T=%d outside 1..%d", T, c->maxT);
     if (!L->router_w || !L->router_scale || !L->shared_blob)
         return fail(MOE_ERR_INVALID_ARG, "layer needs router_w, router_scale and shared_blob");
@@ -842,7 +877,8 @@ extern "C" int moe_ctx_check(moe_ctx* c, moe_stream_t stream) {
     CK(cudaMemset(c->ysh, 0, (size_t)c->cfg.hidden * sizeof(unsigned long long)));
     CK(cudaMemset(c->shared_tag, 0, sizeof(unsigned long long)));
     for (int m = 0; m < 4; m++) c->fparity[m] = 0;
-    return fail(st, "a bounded device wait gave up (status %d); counters reset", st);
+    return fail(st, st == MOE_ERR_TIMEOUT ? "a bounded device wait gave up; counters reset"
+                                          : "a device-side cache lookup found the LFU table invalid");
 }
 
 extern "C" int moe_ctx_info(moe_ctx* c, char* buf, int len) {

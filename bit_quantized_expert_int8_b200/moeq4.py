@@ -25,6 +25,7 @@ MOE_ERR_CUDA = -4
 MOE_ERR_TIMEOUT = -5
 MOE_ERR_CACHE_STATE = -6
 MOE_PRENORM = 1
+MOE_DEVICE_FILL = 2
 MOE_MAX_SLOTS = 32
 
 EXPORTS = ("moe_ctx_create", "moe_ctx_destroy", "moe_ctx_check", "moe_ctx_trace", "moe_ctx_info",

@@ -324,8 +324,18 @@ int moe_cache_lookup_lfu(moe_ctx *ctx, MoeLfuTable *table,
  * flags & MOE_PRENORM: `x` is the fp16 residual stream h; the layer input is
  * RMSNorm(h) (unit weight, eps = cfg.rms_eps, exact sum of squares, result
  * rounded to fp16) and afterwards h <- fp16(h + y) in place.
+ *
+ * flags & MOE_DEVICE_FILL (streaming mode): the misses are filled by the GPU
+ * instead of the host ([LH] pipeline steps 3-4, with the read moved from the
+ * host to the device): the cache lookup writes the miss list to device
+ * memory, and a gather kernel on `copy` reads it and copies each missing blob
+ * from host_store (which must be pinned host memory the device can address)
+ * into its slot, while `main` runs the shared expert.  The call then makes no
+ * host wait and returns as soon as the work is queued; it can be captured in
+ * a CUDA graph.  A table made invalid by an earlier failed host fill makes
+ * the layer compute with slot 0 and moe_ctx_check report MOE_ERR_CACHE_STATE.
  */
-enum { MOE_PRENORM = 1 };
+enum { MOE_PRENORM = 1, MOE_DEVICE_FILL = 2 };
 
 typedef struct {
     const int8_t *router_w;       /* device int8 [E][H] */

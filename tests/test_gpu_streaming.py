@@ -2,6 +2,10 @@
 16 cache slots per layer, 4 layers with skewed router bias N(0, 1.5), 64
 tokens decoded one after another with RMSNorm and the fp16 residual.
 
+Both ways of filling a miss are covered: copies issued by the host after it
+reads the miss list, and MOE_DEVICE_FILL, where a kernel reads the miss list
+in device memory and pulls the blobs from pinned host memory.
+
 Checks (the streaming configuration of the benchmark, at fewer layers and
 tokens so that the oracle finishes in seconds):
 - streaming output equals resident output bit for bit at every layer and
@@ -55,7 +59,9 @@ def stack():
     return out
 
 
-def test_streaming_equals_resident_bitwise(stack):
+@pytest.mark.parametrize("fill", ["host", "device"])
+def test_streaming_equals_resident_bitwise(stack, fill):
+    flags = moeq4.MOE_PRENORM | (moeq4.MOE_DEVICE_FILL if fill == "device" else 0)
     ctx = moeq4.Context(CFG, 1)
     cs = torch.cuda.Stream()
     for s in stack:
@@ -67,7 +73,7 @@ def test_streaming_equals_resident_bitwise(stack):
     for t in range(T):
         for s in stack:
             moeq4.moe_layer_decode(ctx, s["st"], h_st[t:t + 1], 1, y_st,
-                                   flags=moeq4.MOE_PRENORM, copy_stream=cs)
+                                   flags=flags, copy_stream=cs)
             moeq4.moe_layer_decode(ctx, s["rs"], h_rs[t:t + 1], 1, y_rs,
                                    flags=moeq4.MOE_PRENORM)
             torch.cuda.synchronize()
@@ -81,7 +87,9 @@ def test_streaming_equals_resident_bitwise(stack):
     ctx.close()
 
 
-def test_streaming_oracle_forced_cache_and_outputs(stack):
+@pytest.mark.parametrize("fill", ["host", "device"])
+def test_streaming_oracle_forced_cache_and_outputs(stack, fill):
+    flags = moeq4.MOE_PRENORM | (moeq4.MOE_DEVICE_FILL if fill == "device" else 0)
     ctx = moeq4.Context(CFG, 1)
     cs = torch.cuda.Stream()
     for s in stack:
@@ -100,7 +108,7 @@ def test_streaming_oracle_forced_cache_and_outputs(stack):
             so_ref, _ = caches[l].token(ref["idx"])
             hg = torch.from_numpy(h_or.view(np.int16).copy()).view(torch.float16).to(DEV)[None]
             moeq4.moe_layer_decode(ctx, s["st"], hg, 1, y, idx, slot_of=so, x_norm=xn,
-                                   flags=moeq4.MOE_PRENORM, copy_stream=cs)
+                                   flags=flags, copy_stream=cs)
             torch.cuda.synchronize()
             np.testing.assert_array_equal(np_of(xn)[0], x_or)
             assert idx[0].cpu().tolist() == ref["idx"].tolist(), (t, l)
