@@ -77,8 +77,8 @@ def _load():
     lib.oracle_residual_add.restype = None
     lib.oracle_lfu_token.argtypes = [i32, P, P, P, P, P, i32, P, P, P, P, P, P]
     lib.oracle_lfu_token.restype = i32
-    lib.oracle_lfu_unit.argtypes = [i32, P, P, P, P, P, i32, i32, P, P, P, P, P, P]
-    lib.oracle_lfu_unit.restype = i32
+    lib.oracle_lfu_chunk.argtypes = [i32, P, P, P, P, P, i32, i32, P, P, P, P, P, P, P, P, P]
+    lib.oracle_lfu_chunk.restype = i32
     lib.oracle_set_threads.argtypes = [i32]
     lib.oracle_set_threads.restype = i32
     _lib = lib
@@ -250,40 +250,25 @@ class LfuCache:
         n = int(nm[0])
         return slot_of, list(zip(me[:n].tolist(), ms[:n].tolist()))
 
-    def unit(self, idx):
-        """Look up one unit of consecutive tokens (``idx`` [n_tok, k]) at once
-        (``oracle_lfu_unit``); returns (slot_of [n_tok, k], [(expert, slot)])."""
-        idx = _c(np.asarray(idx, np.int32).reshape(-1, np.asarray(idx).shape[-1]), np.int32)
-        n_tok, k = idx.shape
-        slot_of = np.full((n_tok, k), -1, np.int32)
-        me = np.zeros(self.S, np.int32)
-        ms = np.zeros(self.S, np.int32)
-        nm = np.zeros(1, np.int32)
-        rc = _load().oracle_lfu_unit(self.S, _p(self.expert), _p(self.count),
-                                     _p(self.seq), _p(self.counter), _p(idx), n_tok, k,
-                                     _p(slot_of), _p(me), _p(ms), _p(nm),
-                                     _p(self.hits), _p(self.misses))
-        if rc != 0:
-            raise ValueError("oracle_lfu_unit: unit does not fit, repeated expert or bad size")
-        n = int(nm[0])
-        return slot_of, list(zip(me[:n].tolist(), ms[:n].tolist()))
-
     def chunk(self, idx):
-        """A chunk of tokens (``idx`` [T, k]) in units: each unit is the
-        longest run of consecutive tokens, from the first token not yet
-        served, whose distinct experts fit in the S slots.  Returns
-        [(t0, t1, slot_of [t1 - t0, k], [(expert, slot)])] in unit order."""
-        idx = np.asarray(idx, np.int32)
-        T = idx.shape[0]
-        out = []
-        t0 = 0
-        while t0 < T:
-            seen = set(idx[t0].tolist())
-            t1 = t0 + 1
-            while t1 < T and len(seen | set(idx[t1].tolist())) <= self.S:
-                seen |= set(idx[t1].tolist())
-                t1 += 1
-            slot_of, miss = self.unit(idx[t0:t1])
-            out.append((t0, t1, slot_of, miss))
-            t0 = t1
-        return out
+        """Look up a chunk of tokens (``idx`` [T, k]) at once, expert by
+        expert in batches that fit the slots (``oracle_lfu_chunk``).  Returns
+        (slot_of [T, k], batch_of [T, k], [(batch, expert, slot)], n_batch)."""
+        idx = _c(np.asarray(idx, np.int32).reshape(-1, np.asarray(idx).shape[-1]), np.int32)
+        T, k = idx.shape
+        slot_of = np.full((T, k), -1, np.int32)
+        batch_of = np.full((T, k), -1, np.int32)
+        n_max = T * k
+        mb = np.zeros(n_max, np.int32)
+        me = np.zeros(n_max, np.int32)
+        ms = np.zeros(n_max, np.int32)
+        nm = np.zeros(1, np.int32)
+        nb = np.zeros(1, np.int32)
+        rc = _load().oracle_lfu_chunk(self.S, _p(self.expert), _p(self.count),
+                                      _p(self.seq), _p(self.counter), _p(idx), T, k,
+                                      _p(slot_of), _p(batch_of), _p(mb), _p(me), _p(ms),
+                                      _p(nm), _p(nb), _p(self.hits), _p(self.misses))
+        if rc != 0:
+            raise ValueError("oracle_lfu_chunk: repeated expert, S <= k or bad size")
+        n = int(nm[0])
+        return slot_of, batch_of, list(zip(mb[:n].tolist(), me[:n].tolist(), ms[:n].tolist())), int(nb[0])

@@ -449,43 +449,48 @@ int oracle_lfu_token(int S, int32_t *slot_expert, int64_t *slot_count,
     return 0;
 }
 
-/* One unit of a chunk (several consecutive tokens processed at once,
- * chunked prefill: [LH] 04 "Chunked Prefill" -- one expert fetched from
- * storage serves every row of the chunk that uses it) in one layer's LFU
- * cache.  The pages fix no rule for a chunk; this is the per-token rule
- * above applied to the unit's set of experts, each weighted by its uses:
- *  (i)  the distinct experts of the unit in ascending id order: a resident
- *       expert is a hit and its count grows by the number of the unit's
- *       (token, choice) pairs that use it;
- *  (ii) then each missing expert in ascending id order: the lowest-index
- *       empty slot if any, else, among the slots the unit does not use, the
- *       lowest count, ties to the oldest insertion; the newcomer's count is
- *       its number of uses and it takes the next sequence number.
- * Hits and misses count distinct experts of the unit (a miss is one copy).
- * With one token per unit this is exactly oracle_lfu_token.
- * idx is [n_tok][k]; slot_of[t * k + j] is the slot of idx[t * k + j]; the
- * misses are listed in insertion order.  Returns 0, or -1 when the unit's
- * experts do not fit in S slots, an expert repeats within a token, or the
- * sizes are out of range. */
-int oracle_lfu_unit(int S, int32_t *slot_expert, int64_t *slot_count,
-                    int64_t *slot_seq, int64_t *seq_counter,
-                    const int32_t *idx, int n_tok, int k, int32_t *slot_of,
-                    int32_t *miss_expert, int32_t *miss_slot,
-                    int32_t *n_miss, int64_t *hits, int64_t *misses)
+/* A chunk of n_tok tokens (chunked prefill, [LH] 04 "Chunked Prefill": one
+ * expert fetched from storage serves every row of the chunk that uses it) in
+ * one layer's LFU cache.  The pages fix no rule for a chunk; this applies the
+ * per-token rule above to the chunk's distinct experts, each weighted by its
+ * uses, and serves them in batches that fit the slots, so that each expert is
+ * copied at most once per chunk:
+ *  (i)   the distinct experts in ascending id order: a resident expert is a
+ *        hit, its count grows by its number of (token, choice) pairs in the
+ *        chunk, and its slot is pinned to batch 0;
+ *  (ii)  then each missing expert in ascending id order takes the lowest-index
+ *        empty slot if any, else, among the slots not pinned by the current
+ *        batch, the lowest count, ties to the oldest insertion; when every
+ *        slot is pinned, the current batch is complete (its pairs are served
+ *        from the slots), the next batch starts and no slot is pinned; the
+ *        newcomer's count is its number of uses and it takes the next
+ *        sequence number;
+ *  (iii) hits and misses count distinct experts (a miss is one copy).
+ * With one token per chunk (k < S) there is one batch and this is exactly
+ * oracle_lfu_token.  idx is [n_tok][k]; slot_of[q] and batch_of[q] are the
+ * slot and batch of pair q = t * k + j; the misses (batch, expert, slot) are
+ * listed in insertion order; *n_batch is the number of batches.  Returns 0,
+ * or -1 when an expert repeats within a token or the sizes are out of range. */
+int oracle_lfu_chunk(int S, int32_t *slot_expert, int64_t *slot_count,
+                     int64_t *slot_seq, int64_t *seq_counter,
+                     const int32_t *idx, int n_tok, int k, int32_t *slot_of,
+                     int32_t *batch_of, int32_t *miss_batch, int32_t *miss_expert,
+                     int32_t *miss_slot, int32_t *n_miss, int32_t *n_batch,
+                     int64_t *hits, int64_t *misses)
 {
-    int32_t ex[256];
-    int64_t uses[256];
-    int32_t slot_ex[256];
-    char used[256];
+    enum { kMaxDistinct = 4096 };
+    static int32_t ex[kMaxDistinct], slot_ex[kMaxDistinct], batch_ex[kMaxDistinct];
+    static int64_t uses[kMaxDistinct];
+    char pinned[256];
     int nu = 0;
-    if (k < 1 || k > 64 || S < 1 || S > 256 || n_tok < 1)
+    if (k < 1 || k > 64 || S < 1 || S > 256 || S <= k || n_tok < 1)
         return -1;
     for (int t = 0; t < n_tok; t++)
         for (int a = 0; a < k; a++)
             for (int b = a + 1; b < k; b++)
                 if (idx[t * k + a] == idx[t * k + b])
                     return -1;
-    /* distinct experts of the unit and their uses, ascending */
+    /* distinct experts of the chunk and their uses, ascending */
     for (int q = 0; q < n_tok * k; q++) {
         int32_t e = idx[q];
         int i = 0;
@@ -495,7 +500,7 @@ int oracle_lfu_unit(int S, int32_t *slot_expert, int64_t *slot_count,
             uses[i] += 1;
             continue;
         }
-        if (nu == S)
+        if (nu == kMaxDistinct)
             return -1;
         for (int m = nu; m > i; m--) {
             ex[m] = ex[m - 1];
@@ -505,55 +510,65 @@ int oracle_lfu_unit(int S, int32_t *slot_expert, int64_t *slot_count,
         uses[i] = 1;
         nu++;
     }
-    memset(used, 0, sizeof(used));
+    memset(pinned, 0, sizeof(pinned));
     for (int i = 0; i < nu; i++) {
         slot_ex[i] = -1;
+        batch_ex[i] = 0;
         for (int s = 0; s < S; s++)
             if (slot_expert[s] == ex[i]) {
                 slot_count[s] += uses[i];
-                used[s] = 1;
+                pinned[s] = 1;
                 slot_ex[i] = s;
                 *hits += 1;
                 break;
             }
     }
+    int batch = 0;
     *n_miss = 0;
     for (int i = 0; i < nu; i++) {
         if (slot_ex[i] >= 0)
             continue;
         int victim = -1;
-        for (int s = 0; s < S; s++)
-            if (slot_expert[s] < 0) {
-                victim = s;
-                break;
+        for (int pass = 0; pass < 2 && victim < 0; pass++) {
+            if (pass == 1) {             /* every slot pinned: next batch */
+                batch += 1;
+                memset(pinned, 0, sizeof(pinned));
             }
-        if (victim < 0)
-            for (int s = 0; s < S; s++) {
-                if (used[s])
-                    continue;
-                if (victim < 0 || slot_count[s] < slot_count[victim] ||
-                    (slot_count[s] == slot_count[victim] &&
-                     slot_seq[s] < slot_seq[victim]))
+            for (int s = 0; s < S; s++)
+                if (slot_expert[s] < 0) {
                     victim = s;
-            }
-        if (victim < 0)
-            return -1;
+                    break;
+                }
+            if (victim < 0)
+                for (int s = 0; s < S; s++) {
+                    if (pinned[s])
+                        continue;
+                    if (victim < 0 || slot_count[s] < slot_count[victim] ||
+                        (slot_count[s] == slot_count[victim] &&
+                         slot_seq[s] < slot_seq[victim]))
+                        victim = s;
+                }
+        }
         *seq_counter += 1;
         slot_expert[victim] = ex[i];
         slot_count[victim] = uses[i];
         slot_seq[victim] = *seq_counter;
-        used[victim] = 1;
+        pinned[victim] = 1;
         slot_ex[i] = victim;
+        batch_ex[i] = batch;
+        miss_batch[*n_miss] = batch;
         miss_expert[*n_miss] = ex[i];
         miss_slot[*n_miss] = victim;
         *n_miss += 1;
         *misses += 1;
     }
+    *n_batch = batch + 1;
     for (int q = 0; q < n_tok * k; q++) {
         int i = 0;
         while (ex[i] != idx[q])
             i++;
         slot_of[q] = slot_ex[i];
+        batch_of[q] = batch_ex[i];
     }
     return 0;
 }

@@ -442,8 +442,10 @@ def test_lfu_rejects_impossible_requests():
 
 # ------------------------------------------------------ LFU over chunks --
 def _read_chunk_trace(path):
-    """[(chunk rows, [(t0, t1, slot states)])] from the golden chunk trace."""
+    """[(chunk rows, n_batch, [(batch, expert, slot)], slot states)] from the
+    golden chunk trace."""
     out = []
+    rows = None
     with open(path) as f:
         for line in f:
             line = line.split("#")[0].strip()
@@ -451,13 +453,17 @@ def _read_chunk_trace(path):
                 continue
             if line.startswith("chunk"):
                 rows = [[int(v) for v in tok.split()] for tok in line[len("chunk"):].split(";")]
-                out.append((rows, []))
             else:
-                head, slots = line.split("|")
-                _, t0, t1 = head.split()
+                head, miss, slots = line.split("|")
+                nb = int(head.split()[1])
+                ms = []
+                for tok in miss.split():
+                    b, rest = tok.split(":")
+                    e, sl = rest.split(">")
+                    ms.append((int(b), int(e), int(sl)))
                 st = [None if tok == "-" else tuple(int(v) for v in tok.split("."))
                       for tok in slots.split()]
-                out[-1][1].append((int(t0), int(t1), st))
+                out.append((rows, nb, ms, st))
     return out
 
 
@@ -467,56 +473,56 @@ def _state(c):
 
 
 def test_lfu_chunk_hand_trace_golden():
-    """The chunk rule against the hand-derived trace: unit boundaries and the
-    slot contents after every unit."""
+    """The chunk rule against the hand-derived trace: batches, misses in
+    insertion order and the slot contents after every chunk."""
     c = oracle.LfuCache(4)
-    for rows, units in _read_chunk_trace(os.path.join(GOLDEN, "lfu_chunk_trace_s4_k2.txt")):
-        got_units = []
-        snap = oracle.LfuCache(4)
-        snap.expert[:], snap.count[:], snap.seq[:] = c.expert, c.count, c.seq
-        snap.counter[:], snap.hits[:], snap.misses[:] = c.counter, c.hits, c.misses
-        for (t0, t1, _, _) in c.chunk(np.array(rows, np.int32)):
-            # replay unit by unit on the snapshot to see the state after each
-            snap.unit(np.array(rows[t0:t1], np.int32))
-            got_units.append((t0, t1, _state(snap)))
-        assert got_units == units, (rows, got_units, units)
-    assert int(c.hits[0]) == 9 and int(c.misses[0]) == 12
+    for rows, nb, ms, st in _read_chunk_trace(os.path.join(GOLDEN, "lfu_chunk_trace_s4_k2.txt")):
+        slot_of, batch_of, miss, n_batch = c.chunk(np.array(rows, np.int32))
+        assert (n_batch, miss, _state(c)) == (nb, ms, st), rows
+    assert int(c.hits[0]) == 5 and int(c.misses[0]) == 12
 
 
 class NaiveChunkLfu(NaiveLfu):
-    """Independent model of the unit rule: distinct experts with use counts,
-    hits add the uses, newcomers start at their uses."""
+    """Independent model of the chunk rule: distinct experts with their uses,
+    pinned slots as a Python set, a new batch when no slot is free."""
 
-    def unit(self, rows):
+    def chunk(self, rows):
         uses = {}
         for r in rows:
             for e in r:
                 uses[e] = uses.get(e, 0) + 1
-        where = {}
+        where, batch_e = {}, {}
         resident = {en["e"]: s for s, en in enumerate(self.entries) if en}
+        pinned = set()
         for e in sorted(uses):
             if e in resident:
                 s = resident[e]
                 self.entries[s]["n"] += uses[e]
-                where[e] = s
+                where[e], batch_e[e] = s, 0
+                pinned.add(s)
                 self.hits += 1
+        batch, misses = 0, []
         for e in sorted(uses):
             if e in where:
                 continue
             empty = [s for s in range(self.S) if self.entries[s] is None]
-            if empty:
-                s = empty[0]
-            else:
-                cand = [s for s in range(self.S) if s not in where.values()]
-                s = min(cand, key=lambda s: (self.entries[s]["n"], self.entries[s]["t"]))
+            cand = [s for s in range(self.S) if s not in pinned]
+            if not empty and not cand:
+                batch += 1
+                pinned = set()
+                cand = list(range(self.S))
+            s = empty[0] if empty else min(cand, key=lambda s: (self.entries[s]["n"], self.entries[s]["t"]))
             self.t += 1
             self.entries[s] = {"e": e, "n": uses[e], "t": self.t}
-            where[e] = s
+            where[e], batch_e[e] = s, batch
+            pinned.add(s)
+            misses.append((batch, e, s))
             self.misses += 1
-        return [[where[e] for e in r] for r in rows]
+        return ([[where[e] for e in r] for r in rows], [[batch_e[e] for e in r] for r in rows],
+                misses, batch + 1)
 
 
-def test_lfu_chunk_matches_naive_model_and_units_are_maximal():
+def test_lfu_chunk_matches_naive_model():
     rng = np.random.default_rng(21)
     for trial in range(30):
         k = int(rng.integers(1, 9))
@@ -525,39 +531,38 @@ def test_lfu_chunk_matches_naive_model_and_units_are_maximal():
         c, n = oracle.LfuCache(S), NaiveChunkLfu(S)
         for step in range(12):
             T = int(rng.integers(1, 40))
-            # skewed choices, so units hold several tokens
-            p = 1.0 / (1.0 + np.arange(E)) ** 1.2
+            p = 1.0 / (1.0 + np.arange(E)) ** 1.2          # skewed choices
             p /= p.sum()
             rows = np.stack([rng.choice(E, size=k, replace=False, p=p) for _ in range(T)]).astype(np.int32)
-            units = c.chunk(rows)
-            assert units[0][0] == 0 and units[-1][1] == T
-            for (t0, t1, slot_of, miss), nxt in zip(units, units[1:] + [None]):
-                seen = set(rows[t0:t1].ravel().tolist())
-                assert len(seen) <= S                            # the unit fits
-                if nxt is not None:                               # and is maximal
-                    assert nxt[0] == t1
-                    assert len(seen | set(rows[t1].tolist())) > S
-                assert slot_of.tolist() == n.unit(rows[t0:t1].tolist())
+            slot_of, batch_of, miss, nb = c.chunk(rows)
+            n_slot, n_batch_of, n_miss, n_nb = n.chunk(rows.tolist())
+            assert slot_of.tolist() == n_slot and batch_of.tolist() == n_batch_of
+            assert miss == n_miss and nb == n_nb
+            # every expert of the chunk is copied at most once, and a batch
+            # never holds more experts than slots
+            assert len({e for _, e, _ in miss}) == len(miss)
+            for b in range(nb):
+                assert len({int(e) for e in rows[batch_of == b]}) <= S
         assert (int(c.hits[0]), int(c.misses[0])) == (n.hits, n.misses)
 
 
-def test_lfu_one_token_units_are_the_token_rule():
-    """A unit of one token is the per-token rule exactly (same slots, counts,
-    insertion numbers and totals)."""
+def test_lfu_one_token_chunks_are_the_token_rule():
+    """A chunk of one token is the per-token rule exactly (one batch; same
+    slots, counts, insertion numbers and totals)."""
     rng = np.random.default_rng(5)
     a, b = oracle.LfuCache(16), oracle.LfuCache(16)
     for t in range(400):
         idx = rng.choice(128, size=8, replace=False).astype(np.int32)
         sa, ma = a.token(idx)
-        sb, mb = b.unit(idx[None, :])
-        assert sa.tolist() == sb[0].tolist() and ma == mb
+        sb, bb, mb, nb = b.chunk(idx[None, :])
+        assert sa.tolist() == sb[0].tolist() and nb == 1
+        assert ma == [(e, s) for _, e, s in mb]
     assert _state(a) == _state(b)
     assert (int(a.hits[0]), int(a.misses[0])) == (int(b.hits[0]), int(b.misses[0]))
 
 
-def test_lfu_unit_rejects_units_that_do_not_fit():
-    c = oracle.LfuCache(4)
+def test_lfu_chunk_rejects_bad_requests():
     with pytest.raises(ValueError):
-        c.unit(np.array([[1, 2], [3, 4], [5, 6]], np.int32))   # 6 experts > 4 slots
+        oracle.LfuCache(2).chunk(np.array([[1, 2]], np.int32))      # S <= k
     with pytest.raises(ValueError):
-        c.unit(np.array([[7, 7]], np.int32))
+        oracle.LfuCache(8).chunk(np.array([[7, 7]], np.int32))
