@@ -50,9 +50,11 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=15.0)
     p.add_argument("--batch-sizes", default="1,8,32,64,128,256",
                    help="tokens per step of the batched sweep (comma-separated)")
-    p.add_argument("--workload", choices=("stack", "streaming", "batched"), default="stack",
+    p.add_argument("--chunk", type=int, default=128, help="prefill chunk (tokens)")
+    p.add_argument("--workload", choices=("stack", "streaming", "batched", "prefill"), default="stack",
                    help="stack (default, the headline line), streaming (experts in pinned host "
-                        "memory behind the LFU cache) or batched (one layer, T tokens per step)")
+                        "memory behind the LFU cache), batched (one layer, T tokens per step) or "
+                        "prefill (streaming, the prompt in chunks)")
     return p.parse_args()
 
 
@@ -516,6 +518,94 @@ def run_streaming(args):
             "h2d_link_gbs_measured": round(link, 2)}), flush=True)
 
 
+def run_prefill(args):
+    """Chunked prefill in streaming mode: a 512-token prompt through the 30-layer
+    stack in chunks of 128 tokens (chunk-major: each chunk through every layer),
+    every routed expert in pinned host memory behind a 16-slot LFU cache per
+    layer (cold at the start of each step).  A chunk is one cache lookup and
+    one copy per missing expert per unit of tokens whose experts fit the
+    slots.  Reports prompt tokens/s, bytes copied per prompt token and the
+    hit rate (distinct experts per unit), for host- and device-issued fills."""
+    import torch
+
+    from bit_quantized_expert_int8_b200 import moeq4, synth
+    from bit_quantized_expert_int8_b200.config import LAYER
+    cfg = LAYER
+    L = args.layers
+    P = 512 if args.tokens == N_TOKENS else args.tokens
+    C = args.chunk
+    dev = torch.device("cuda", 0)
+    moeq4.load()
+    nb = synth.blob_bytes(cfg.H, cfg.I)
+    layers, keep = [], []
+    for l in range(L):
+        d = synth.layer_weights(cfg, SEED, l, dev, bias_std=BIAS_STD)
+        store = torch.empty((cfg.E, nb), dtype=torch.uint8, pin_memory=True)
+        store.copy_(d["experts"])
+        del d["experts"]
+        slots = torch.zeros((cfg.S, nb), dtype=torch.uint8, device=dev)
+        table = moeq4.new_lfu_table()
+        layers.append(moeq4.Layer(d["router_w"], d["router_scale"], d["router_bias"], d["shared"],
+                                  None, store, slots, table))
+        keep.append((d, store, slots, table))
+    torch.cuda.empty_cache()
+    ctx = moeq4.Context(cfg, C)
+    copy_stream = torch.cuda.Stream()
+    h0 = synth.tokens(P, cfg.H, SEED + 1, dev)
+    h = h0.clone()
+    y = torch.empty((C, cfg.H), dtype=torch.float32, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for fill in ("host", "device"):
+        flags = moeq4.MOE_PRENORM | (moeq4.MOE_DEVICE_FILL if fill == "device" else 0)
+
+        def step():
+            for (_, _, _, table) in keep:
+                moeq4.moe_lfu_init(ctx, table, cfg.S)
+            h.copy_(h0)
+            for c0 in range(0, P, C):
+                n = min(C, P - c0)
+                for lay in layers:
+                    moeq4.moe_layer_decode(ctx, lay, h[c0:c0 + n], n, y[:n], flags=flags,
+                                           copy_stream=copy_stream)
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        hits = misses = 0
+        times = []
+        clocks = ClockSampler(0)
+        clocks.start()
+        for _ in range(args.steps):
+            e0.record()
+            step()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+            for (_, _, _, table) in keep:
+                tb = moeq4.read_lfu_table(table)
+                hits += tb.hits
+                misses += tb.misses
+        clk = clocks.stop()
+        moeq4.moe_ctx_check(ctx)
+        ms = statistics.median(times)
+        h2d = misses / args.steps * nb
+        print(json.dumps({
+            "metric": METRIC, "workload": f"prefill{L}x{P}/chunk{C}", "fill": fill,
+            "value": round(P / (ms / 1000.0), 3), "unit": "prompt tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+            "ms_per_step_min_max": [round(min(times), 3), round(max(times), 3)],
+            "timing": f"median of {len(times)} steps", "higher_is_better": True,
+            "config": {"layers": L, "prompt_tokens": P, "chunk": C, "slots": cfg.S,
+                       "order": "each chunk through every layer", "cache": "cold at each step",
+                       "expert_store": "pinned host memory"},
+            "clocks": clk,
+            "hit_rate_distinct_experts": round(hits / max(1, hits + misses), 4),
+            "copies_per_step": int(misses / args.steps),
+            "h2d_bytes_per_step": int(h2d),
+            "h2d_bytes_per_prompt_token": int(h2d / P),
+            "h2d_gbs_over_step": round(h2d / (ms * 1e-3) / 1e9, 2)}), flush=True)
+
+
 def bucket_split(counts, T, min_tokens=4, min_step=32):
     """Experts of one step by the kernel that serves them: `counts` holds the
     pairs routed to each expert.  In steps of at least `min_step` tokens a
@@ -616,6 +706,8 @@ def main():
         run_streaming(args)
     elif args.workload == "batched":
         run_batched(args)
+    elif args.workload == "prefill":
+        run_prefill(args)
     else:
         run_ours(args)
 

@@ -21,17 +21,22 @@ constexpr int kGrpTokens = 4;          // tokens per pass of a grouped kernel
 constexpr int kGrpThreads = 256;
 constexpr int kGrpChunk = 16;          // shared expert: tokens per CTA (grid z splits the step)
 
-// Groups the T*k routed pairs by expert: e_off[E + 1] (prefix counts) and
-// list[T*k] (pair indices q of expert e at e_off[e] .. e_off[e + 1]).  One CTA.
+// Groups the P routed pairs by expert: e_off[E + 1] (prefix counts) and
+// list[P] (pair indices q of expert e at e_off[e] .. e_off[e + 1]).
+// "Experts" may be cache slots (idx = slot_of, E = the slot count); with
+// sel, only the pairs q with sel[q] == sel_val take part (a batch of a
+// streaming chunk).  One CTA.
 __global__ void __launch_bounds__(1024) k_group_pairs(const int32_t* __restrict__ idx, int P, int E,
-                                                      int* __restrict__ e_off, int* __restrict__ list) {
+                                                      int* __restrict__ e_off, int* __restrict__ list,
+                                                      const int32_t* __restrict__ sel = nullptr,
+                                                      int sel_val = 0) {
     __shared__ int cnt[MOE_MAX_EXPERTS + 1];
     const int tid = threadIdx.x;
     for (int e = tid; e <= E; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
     for (int q = tid; q < P; q += blockDim.x) {
         const int e = idx[q];
-        if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+        if (e >= 0 && e < E && (!sel || sel[q] == sel_val)) atomicAdd(&cnt[e], 1);
     }
     __syncthreads();
     if (tid == 0) {
@@ -47,7 +52,7 @@ __global__ void __launch_bounds__(1024) k_group_pairs(const int32_t* __restrict_
     __syncthreads();
     for (int q = tid; q < P; q += blockDim.x) {
         const int e = idx[q];
-        if (e >= 0 && e < E) list[atomicAdd(&cnt[e], 1)] = q;
+        if (e >= 0 && e < E && (!sel || sel[q] == sel_val)) list[atomicAdd(&cnt[e], 1)] = q;
     }
 }
 

@@ -139,6 +139,112 @@ __global__ void k_lfu_lookup(MoeLfuTable* __restrict__ tb, const int32_t* __rest
     *n_miss = nm;
 }
 
+// LFU lookup of a chunk of tokens (chunked prefill: "Gemma 4 26B : Comment
+// faire tourner un LLM en 2 Go de RAM", section 04 "Chunked Prefill" -- one
+// expert fetched into the cache serves every row of the chunk that uses it).
+// The per-token rule of k_lfu_lookup applied to the chunk's distinct experts,
+// each weighted by its uses, served in batches that fit the slots:
+//   - the distinct experts in ascending id order: a resident one is a hit,
+//     its count grows by its number of (token, choice) pairs, and its slot
+//     is pinned to batch 0;
+//   - then each missing one takes the lowest empty slot, else, among the
+//     slots not pinned by the current batch, the lowest count, ties to the
+//     oldest insertion; when every slot is pinned the next batch starts with
+//     no slot pinned; the newcomer starts at its number of uses;
+//   - hits and misses count distinct experts (a miss is one copy).
+// Outputs: slot_of and batch_of [n_tok][k] (device), and in `plan` (ints,
+// mapped host memory) the number of batches nb, then nb + 1 offsets and nb
+// counts into the miss list, then the misses as (expert, slot) pairs in
+// insertion order (batch by batch): plan = [nb, off[0..max_b], cnt[0..max_b),
+// pairs...] with max_b = n_experts + 1.  An invalid table gives nb = -1, slot
+// 0 everywhere and MOE_ERR_CACHE_STATE in the status word.  One thread.
+__global__ void k_lfu_chunk(MoeLfuTable* __restrict__ tb, const int32_t* __restrict__ idx, int n_tok,
+                            int k, int n_experts, int32_t* __restrict__ slot_of,
+                            int32_t* __restrict__ batch_of, int32_t* __restrict__ plan,
+                            int* __restrict__ status) {
+    if (threadIdx.x != 0) return;
+    const int P = n_tok * k, max_b = n_experts + 1;
+    int32_t* off = plan + 1;
+    int32_t* cnt = off + max_b + 1;
+    int32_t* pairs = cnt + max_b;
+    if (!tb->valid) {
+        for (int q = 0; q < P; q++) { slot_of[q] = 0; batch_of[q] = 0; }
+        if (status) atomicCAS(status, 0, MOE_ERR_CACHE_STATE);
+        __threadfence_system();
+        plan[0] = -1;
+        return;
+    }
+    const int S = tb->n_slots;
+    // uses per expert id (n_experts <= MOE_MAX_EXPERTS), then slot and batch per id
+    int uses[MOE_MAX_EXPERTS], where[MOE_MAX_EXPERTS], bat[MOE_MAX_EXPERTS];
+    for (int e = 0; e < n_experts; e++) { uses[e] = 0; where[e] = -1; bat[e] = 0; }
+    for (int q = 0; q < P; q++) {
+        const int e = idx[q];
+        if (e < 0 || e >= n_experts) {           // not a routing: refuse the chunk
+            for (int r = 0; r < P; r++) { slot_of[r] = 0; batch_of[r] = 0; }
+            if (status) atomicCAS(status, 0, MOE_ERR_CACHE_STATE);
+            __threadfence_system();
+            plan[0] = -1;
+            return;
+        }
+        uses[e] += 1;
+    }
+    uint32_t pinned = 0;
+    for (int e = 0; e < n_experts; e++) {
+        if (!uses[e]) continue;
+        for (int s = 0; s < S; s++)
+            if (tb->expert[s] == e) {
+                tb->count[s] += uses[e];
+                pinned |= 1u << s;
+                where[e] = s;
+                tb->hits += 1;
+                break;
+            }
+    }
+    int batch = 0, nm = 0;
+    off[0] = 0;
+    for (int e = 0; e < n_experts; e++) {
+        if (!uses[e] || where[e] >= 0) continue;
+        int v = -1;
+        for (int pass = 0; pass < 2 && v < 0; pass++) {
+            if (pass == 1) {                     // every slot pinned: the next batch
+                cnt[batch] = nm - off[batch];
+                batch += 1;
+                off[batch] = nm;
+                pinned = 0;
+            }
+            for (int s = 0; s < S && v < 0; s++)
+                if (tb->expert[s] < 0) v = s;
+            if (v < 0)
+                for (int s = 0; s < S; s++) {
+                    if (pinned & (1u << s)) continue;
+                    if (v < 0 || tb->count[s] < tb->count[v] ||
+                        (tb->count[s] == tb->count[v] && tb->seq[s] < tb->seq[v]))
+                        v = s;
+                }
+        }
+        tb->counter += 1;
+        tb->expert[v] = e;
+        tb->count[v] = uses[e];
+        tb->seq[v] = tb->counter;
+        pinned |= 1u << v;
+        where[e] = v;
+        bat[e] = batch;
+        pairs[2 * nm] = e;
+        pairs[2 * nm + 1] = v;
+        nm++;
+        tb->misses += 1;
+    }
+    cnt[batch] = nm - off[batch];
+    off[batch + 1] = nm;
+    for (int q = 0; q < P; q++) {
+        slot_of[q] = where[idx[q]];
+        batch_of[q] = bat[idx[q]];
+    }
+    __threadfence_system();
+    plan[0] = batch + 1;
+}
+
 // Device-initiated cache fill: the blobs of the miss list, copied from pinned
 // host memory (read over the bus by plain 16-byte loads) into their cache
 // slots, with no host involvement ("Gemma 4 26B : Comment faire tourner un LLM

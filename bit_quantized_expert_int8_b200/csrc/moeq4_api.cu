@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -87,7 +88,10 @@ struct moe_ctx {
     int32_t* n_miss_d = nullptr;
     int32_t* n_miss_host = nullptr;
     int32_t* n_miss_dev = nullptr;
-    cudaEvent_t ev_lookup = nullptr, ev_copy = nullptr;
+    cudaEvent_t ev_lookup = nullptr, ev_copy = nullptr, ev_ffn = nullptr;
+    int32_t* plan_host = nullptr;    // mapped pinned: a streaming chunk's batch plan (k_lfu_chunk)
+    int32_t* plan_dev = nullptr;
+    int32_t* batch_of = nullptr;     // [maxT * k] batch of every routed pair of a streaming chunk
     cudaStream_t cap_stream = nullptr;
     // stack graph
     cudaGraphExec_t stack_exec = nullptr;
@@ -179,6 +183,8 @@ extern "C" int moe_ctx_destroy(moe_ctx* c) {
     if (c->stack_exec) cudaGraphExecDestroy(c->stack_exec);
     if (c->ev_lookup) cudaEventDestroy(c->ev_lookup);
     if (c->ev_copy) cudaEventDestroy(c->ev_copy);
+    if (c->ev_ffn) cudaEventDestroy(c->ev_ffn);
+    if (c->plan_host) cudaFreeHost(c->plan_host);
     if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
     if (c->miss_host) cudaFreeHost(c->miss_host);
     if (c->ws) cudaFree(c->ws);
@@ -337,6 +343,7 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     size_t o_y = take(P * H * sizeof(float));
     size_t o_xn = take(T * H * sizeof(__half));
     size_t o_slot = take(T * k * sizeof(int32_t));
+    size_t o_batch = take(T * k * sizeof(int32_t));
     size_t o_cur = take(sizeof(int));
     size_t o_hcur = take(H * sizeof(__half));
     size_t o_ycur = take(H * sizeof(float));
@@ -347,7 +354,8 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     size_t o_halt = take(H * sizeof(__half));
     size_t o_dlimb = take((k * (size_t)cfg->inter + cfg->inter_shared) / 32 * kDLimbWords * 4);
     size_t o_ysh = take(H * sizeof(unsigned long long));
-    size_t o_eoff = take((E + 1) * sizeof(int));
+    // buckets are experts, or cache slots for a streaming chunk
+    size_t o_eoff = take(((E > MOE_MAX_SLOTS ? E : MOE_MAX_SLOTS) + 1) * sizeof(int));
     size_t o_plist = take(T * k * sizeof(int));
     size_t o_hpl = take(2 * P * (size_t)c->maxI * sizeof(__nv_bfloat16));   // h hi / lo planes
     size_t o_xs = take(P * H * sizeof(__half));                              // x rows, bucket order
@@ -375,6 +383,7 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
         c->y_pairs = (float*)(c->ws + o_y);
         c->x_norm = (__half*)(c->ws + o_xn);
         c->slot_of = (int32_t*)(c->ws + o_slot);
+        c->batch_of = (int32_t*)(c->ws + o_batch);
         c->cursor = (int*)(c->ws + o_cur);
         c->h_cur = (__half*)(c->ws + o_hcur);
         c->y_cur = (float*)(c->ws + o_ycur);
@@ -397,6 +406,10 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
         e = cudaEventCreateWithFlags(&c->ev_lookup, cudaEventDisableTiming);
     }
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_copy, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_ffn, cudaEventDisableTiming);
+    if (e == cudaSuccess)
+        e = cudaHostAlloc((void**)&c->plan_host, (4 * E + 8) * sizeof(int32_t), cudaHostAllocMapped);
+    if (e == cudaSuccess) e = cudaHostGetDevicePointer((void**)&c->plan_dev, c->plan_host, 0);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking);
     const int smem_router = (int)(H * sizeof(long long));
     if (e == cudaSuccess)
@@ -793,6 +806,110 @@ static int layer_streaming_fused(moe_ctx* c, const MoeLayer* L, __half* x, const
     return MOE_OK;
 }
 
+// Streaming chunk of T > 1 tokens (chunked prefill: [LH] 04 "Chunked
+// Prefill" -- one expert fetched into the cache serves every row of the chunk
+// that uses it).  Router for all T tokens, then one cache lookup of the whole
+// chunk (k_lfu_chunk): the chunk's distinct experts are served in batches that
+// fit the slots, each expert copied at most once.  The shared expert runs for
+// all T tokens while the host reads the batch plan (one host wait per chunk).
+// Per batch: one copy per missing blob (host-issued, or the device gather with
+// MOE_DEVICE_FILL), issued after the previous batch's kernels, which may still
+// read the slots they overwrite; then the CUDA-core grouped kernels serve the
+// batch's pairs with the cache slots as the buckets.  Combine and residual for
+// all T tokens at the end.
+static int layer_streaming_chunk(moe_ctx* c, const MoeLayer* L, __half* x, int T, const MoeLayerOut* o,
+                                 int flags, cudaStream_t s, cudaStream_t cs) {
+    const MoeConfig& g = c->cfg;
+    const int k = g.top_k, H = g.hidden, I = g.inter, Is = g.inter_shared, E = g.n_experts;
+    const bool dev_fill = (flags & MOE_DEVICE_FILL) != 0;
+    const size_t stride = BlobLayout(H, I).bytes;
+    const __half* xin = x;
+    __half* xn = o->x_norm ? reinterpret_cast<__half*>(o->x_norm) : c->x_norm;
+    if (flags & MOE_PRENORM) {
+        k_rmsnorm<<<T, 256, 0, s>>>(x, xn, H, g.rms_eps);
+        CKL();
+        xin = xn;
+    }
+    int32_t* idx = o->topk_idx ? o->topk_idx : c->idx;
+    float* w = o->topk_w ? o->topk_w : c->w;
+    int32_t* slot_of = o->slot_of ? o->slot_of : c->slot_of;
+    const void* dstore = nullptr;
+    if (dev_fill) {
+        void* p = nullptr;
+        if (cudaHostGetDevicePointer(&p, const_cast<void*>(L->host_store), 0) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return fail(MOE_ERR_INVALID_ARG, "MOE_DEVICE_FILL needs host_store in pinned host memory "
+                                             "that the device can address");
+        }
+        dstore = p;
+    }
+    TRY(launch_router(c, L->router_w, L->router_scale, L->router_bias, xin, T, idx, w, nullptr, s));
+    k_lfu_chunk<<<1, 32, 0, s>>>(L->lfu, idx, T, k, E, slot_of, c->batch_of, c->plan_dev, c->status);
+    CKL();
+    CK(cudaEventRecord(c->ev_lookup, s));
+    // the shared expert for every token of the chunk, while the host reads
+    // the plan and the first batch's misses are filled
+    const uint8_t* sh = static_cast<const uint8_t*>(L->shared_blob);
+    uint8_t* slots = static_cast<uint8_t*>(L->slots);
+    const uint8_t* store = static_cast<const uint8_t*>(L->host_store);
+    const int chunks = (T + kGrpChunk - 1) / kGrpChunk;
+    k_gateup_grouped<true><<<dim3(Is / 16, 1, chunks), kGrpThreads, grouped_smem_gu(H), s>>>(
+        slots, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, 0x7fffffff, g.gelu, c->h_ws, c->maxI);
+    CKL();
+    k_down_grouped<true><<<dim3(H / 16, 1, chunks), kGrpThreads, grouped_smem_dn(Is), s>>>(
+        slots, stride, sh, H, Is, T, c->e_off, c->plist, 0x7fffffff, c->h_ws, c->maxI, c->y_pairs);
+    CKL();
+    CK(cudaEventSynchronize(c->ev_lookup));
+    const int max_b = E + 1;
+    const int nb = *(volatile int32_t*)c->plan_host;
+    if (nb < 0) return fail(MOE_ERR_CACHE_STATE, "LFU table is invalid (an earlier fill failed)");
+    const int32_t* off = c->plan_host + 1;
+    const int32_t* pairs = c->plan_host + 1 + (max_b + 1) + max_b;
+    for (int b = 0; b < nb; b++) {
+        const int n = off[b + 1] - off[b];
+        // batch b's copies may overwrite slots the previous batch still reads
+        CK(cudaStreamWaitEvent(cs, b > 0 ? c->ev_ffn : c->ev_lookup, 0));
+        if (n > 0) {
+            if (dev_fill) {
+                k_fill_from_host<<<dim3(kFillParts, n), kFillThreads, 0, cs>>>(
+                    static_cast<const uint8_t*>(dstore), slots, stride, c->plan_dev + (pairs - c->plan_host) + 2 * off[b],
+                    c->plan_dev + 1 + (max_b + 1) + b, E, MOE_MAX_SLOTS);
+                CKL();
+            } else {
+                for (int m = off[b]; m < off[b + 1]; m++) {
+                    const int e = pairs[2 * m], sl = pairs[2 * m + 1];
+                    cudaError_t err = cudaSuccess;
+                    if (c->fail_copy_at >= 0 && c->copies_seen == c->fail_copy_at) err = cudaErrorInvalidValue;
+                    c->copies_seen++;
+                    if (err == cudaSuccess)
+                        err = cudaMemcpyAsync(slots + (size_t)sl * stride, store + (size_t)e * stride, stride,
+                                              cudaMemcpyHostToDevice, cs);
+                    if (err != cudaSuccess) {
+                        k_lfu_invalidate<<<1, 1, 0, s>>>(L->lfu);
+                        return fail(MOE_ERR_CACHE_STATE, "fill of expert %d into slot %d failed: %s; table "
+                                    "marked invalid", e, sl, cudaGetErrorString(err));
+                    }
+                }
+            }
+            CK(cudaEventRecord(c->ev_copy, cs));
+            CK(cudaStreamWaitEvent(s, c->ev_copy, 0));
+        }
+        // the batch's routed pairs grouped by cache slot
+        k_group_pairs<<<1, 1024, 0, s>>>(slot_of, T * k, MOE_MAX_SLOTS, c->e_off, c->plist, c->batch_of, b);
+        CKL();
+        k_gateup_grouped<false><<<dim3(I / 16, MOE_MAX_SLOTS), kGrpThreads, grouped_smem_gu(H), s>>>(
+            slots, stride, sh, H, I, xin, T, k, c->e_off, c->plist, 0x7fffffff, g.gelu, c->h_ws, c->maxI);
+        CKL();
+        k_down_grouped<false><<<dim3(H / 16, MOE_MAX_SLOTS), kGrpThreads, grouped_smem_dn(I), s>>>(
+            slots, stride, sh, H, I, T, c->e_off, c->plist, 0x7fffffff, c->h_ws, c->maxI, c->y_pairs);
+        CKL();
+        CK(cudaEventRecord(c->ev_ffn, s));
+    }
+    TRY(launch_combine(c, c->y_pairs + (size_t)T * H, c->y_pairs, w, T, o->y,
+                       (flags & MOE_PRENORM) ? x : nullptr, s));
+    return MOE_OK;
+}
+
 static int layer_streaming(moe_ctx* c, const MoeLayer* L, __half* x, const MoeLayerOut* o,
                            int flags, cudaStream_t s, cudaStream_t cs) {
     if (c->fused_ok) return layer_streaming_fused(c, L, x, o, flags, s, cs);
@@ -848,9 +965,12 @@ extern "C" int moe_layer_decode(moe_ctx* c, const MoeLayer* L, moe_half* x, int 
     }
     if (!L->host_store || !L->slots || !L->lfu || !copy)
         return fail(MOE_ERR_INVALID_ARG, "streaming mode needs host_store, slots, lfu and a copy stream");
-    if (T != 1) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "streaming mode decodes one token per call");
+    if (T > 1 && !c->grouped_ok)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "streaming chunks need the grouped kernels, whose tiles "
+                    "do not fit this shape");
     if (!aligned16(L->slots) || !aligned16(L->lfu) || !aligned16(L->host_store))
         return fail(MOE_ERR_ALIGNMENT, "moe_layer_decode: pointers must be 16-byte aligned");
+    if (T > 1) return layer_streaming_chunk(c, L, reinterpret_cast<__half*>(x), T, o, flags, main, copy);
     return layer_streaming(c, L, reinterpret_cast<__half*>(x), o, flags, main, copy);
 }
 

@@ -310,7 +310,7 @@ int moe_cache_lookup_lfu(moe_ctx *ctx, MoeLfuTable *table,
  * Resident mode (layer->experts != NULL): router, grouped FFN of the shared
  * and the routed experts, combine; all on `main`, no host wait.
  *
- * Streaming mode (layer->experts == NULL; host_store, slots, lfu set; T = 1):
+ * Streaming mode (layer->experts == NULL; host_store, slots, lfu set), T = 1:
  * router and cache lookup on `main`, then the shared-expert FFN on `main`
  * while the host waits for the miss list and issues one cudaMemcpyAsync per
  * missing blob on `copy`; `main` waits for the copies, runs the routed FFN
@@ -320,6 +320,23 @@ int moe_cache_lookup_lfu(moe_ctx *ctx, MoeLfuTable *table,
  * hands its intermediate to the routed part through a tagged word that the
  * routed part waits for (bounded), so a missing shared part ends in
  * MOE_ERR_TIMEOUT from moe_ctx_check rather than in wrong output.
+ *
+ * Streaming mode, 1 < T <= max_tokens (chunked prefill, [LH] 04 "Chunked
+ * Prefill": one expert fetched serves every row of the chunk that uses it):
+ * router for the T tokens, then one LFU lookup of the whole chunk.  The
+ * chunk's distinct experts are served in batches that fit the slots: hits
+ * first (count += their uses in the chunk, slot pinned to batch 0), then each
+ * missing expert in ascending id takes the lowest empty slot, else the
+ * unpinned slot with the lowest count (ties to the oldest insertion), and a
+ * new batch starts, with no slot pinned, when every slot is pinned; a
+ * newcomer's count is its uses; hits and misses count distinct experts.  Each
+ * expert is copied at most once per chunk.  The shared expert runs for all T
+ * tokens while the host reads the batch plan (one host wait per call, in both
+ * fill modes); then per batch the missing blobs are copied (after the
+ * previous batch's kernels) and the grouped kernels serve the batch's
+ * (token, choice) pairs from the slots; combine at the end.  slot_of receives
+ * the slot each pair was served from.  With T = 1 this rule is the per-token
+ * rule above.
  *
  * flags & MOE_PRENORM: `x` is the fp16 residual stream h; the layer input is
  * RMSNorm(h) (unit weight, eps = cfg.rms_eps, exact sum of squares, result
