@@ -51,10 +51,15 @@ def parse():
     p.add_argument("--batch-sizes", default="1,8,32,64,128,256",
                    help="tokens per step of the batched sweep (comma-separated)")
     p.add_argument("--chunk", type=int, default=128, help="prefill chunk (tokens)")
-    p.add_argument("--workload", choices=("stack", "streaming", "batched", "prefill"), default="stack",
+    p.add_argument("--store-dir", default=tempfile.gettempdir(), help="directory of the expert file")
+    p.add_argument("--store-layers", type=int, default=8, help="layers in the expert file")
+    p.add_argument("--store-threads", type=int, default=16, help="pread threads")
+    p.add_argument("--workload", choices=("stack", "streaming", "batched", "prefill", "storage"),
+                   default="stack",
                    help="stack (default, the headline line), streaming (experts in pinned host "
                         "memory behind the LFU cache), batched (one layer, T tokens per step) or "
-                        "prefill (streaming, the prompt in chunks)")
+                        "prefill (streaming, the prompt in chunks) or storage (misses read "
+                        "from an expert file)")
     return p.parse_args()
 
 
@@ -606,6 +611,115 @@ def run_prefill(args):
             "h2d_gbs_over_step": round(h2d / (ms * 1e-3) / 1e9, 2)}), flush=True)
 
 
+def _fs_of(path):
+    """File system type of the mount holding path (from /proc/mounts)."""
+    best, fs = "", "unknown"
+    try:
+        with open("/proc/mounts") as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 3 and os.path.abspath(path).startswith(parts[1]) and len(parts[1]) > len(best):
+                    best, fs = parts[1], parts[2]
+    except OSError:
+        pass
+    return fs
+
+
+def run_storage(args):
+    """The storage tier: the stack's routed experts in an expert file (blobs
+    padded to 4 KiB, read with parallel pread, O_DIRECT where the file system
+    allows), misses read into pinned staging and copied to the 16 slots per
+    layer.  Two lines: decode (tokens one after another) and prefill (the
+    prompt in chunks, each chunk through every layer), cold cache each step."""
+    import torch
+
+    from bit_quantized_expert_int8_b200 import moeq4, synth
+    from bit_quantized_expert_int8_b200.config import LAYER
+    cfg = LAYER
+    L = args.store_layers
+    dev = torch.device("cuda", 0)
+    moeq4.load()
+    nb = synth.blob_bytes(cfg.H, cfg.I)
+    d_all = [synth.layer_weights(cfg, SEED, l, dev, bias_std=BIAS_STD) for l in range(L)]
+    path = os.path.join(args.store_dir, f"moeq4_experts_{os.getpid()}.bin")
+    t0 = time.perf_counter()
+    moeq4.write_expert_file(path, [d["experts"].cpu() for d in d_all], nb)
+    os.sync()
+    write_s = time.perf_counter() - t0
+    fst = moeq4.Store(path, L, cfg.E, nb, n_threads=args.store_threads, n_staging=cfg.S)
+    layers = []
+    for l, d in enumerate(d_all):
+        del d["experts"]
+        slots = torch.zeros((cfg.S, nb), dtype=torch.uint8, device=dev)
+        table = moeq4.new_lfu_table()
+        layers.append((moeq4.Layer(d["router_w"], d["router_scale"], d["router_bias"], d["shared"],
+                                   None, None, slots, table, store=fst, store_layer=l), slots, table))
+    torch.cuda.empty_cache()
+    C = args.chunk
+    ctx = moeq4.Context(cfg, C)
+    copy_stream = torch.cuda.Stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    try:
+        for mode, P in (("decode", 128), ("prefill", 512)):
+            h0 = synth.tokens(P, cfg.H, SEED + 1, dev)
+            h = h0.clone()
+            y = torch.empty((C, cfg.H), dtype=torch.float32, device=dev)
+
+            def step():
+                for (_, _, table) in layers:
+                    moeq4.moe_lfu_init(ctx, table, cfg.S)
+                h.copy_(h0)
+                if mode == "decode":
+                    for t in range(P):
+                        for (lay, _, _) in layers:
+                            moeq4.moe_layer_decode(ctx, lay, h[t:t + 1], 1, y[:1], flags=moeq4.MOE_PRENORM,
+                                                   copy_stream=copy_stream)
+                else:
+                    for c0 in range(0, P, C):
+                        n = min(C, P - c0)
+                        for (lay, _, _) in layers:
+                            moeq4.moe_layer_decode(ctx, lay, h[c0:c0 + n], n, y[:n], flags=moeq4.MOE_PRENORM,
+                                                   copy_stream=copy_stream)
+
+            for _ in range(args.warmup):
+                step()
+            torch.cuda.synchronize()
+            b0, s0, direct = fst.stats()
+            misses = 0
+            times = []
+            clocks = ClockSampler(0)
+            clocks.start()
+            for _ in range(args.steps):
+                e0.record()
+                step()
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1))
+                misses += sum(moeq4.read_lfu_table(t).misses for (_, _, t) in layers)
+            clk = clocks.stop()
+            moeq4.moe_ctx_check(ctx)
+            b1, s1, direct = fst.stats()
+            ms = statistics.median(times)
+            print(json.dumps({
+                "metric": METRIC, "workload": f"storage-{mode}{L}x{P}", "value": round(P / (ms / 1000.0), 3),
+                "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(ms, 3), "ms_per_step_min_max": [round(min(times), 3), round(max(times), 3)],
+                "timing": f"median of {len(times)} steps", "higher_is_better": True,
+                "config": {"layers": L, "tokens": P, "chunk": C if mode == "prefill" else 1, "slots": cfg.S,
+                           "expert_store": "file", "file_system": _fs_of(path), "o_direct": bool(direct),
+                           "reader_threads": args.store_threads, "cache": "cold at each step",
+                           "file_bytes": os.path.getsize(path), "file_write_s": round(write_s, 2)},
+                "clocks": clk,
+                "copies_per_step": int(misses / args.steps),
+                "read_bytes_per_step": int((b1 - b0) / args.steps),
+                "read_gbs_while_reading": round((b1 - b0) / max(1e-9, s1 - s0) / 1e9, 2),
+                "read_gbs_over_step": round((b1 - b0) / args.steps / (ms * 1e-3) / 1e9, 2),
+                "read_bytes_per_token": int((b1 - b0) / args.steps / P)}), flush=True)
+    finally:
+        fst.close()
+        os.unlink(path)
+
+
 def bucket_split(counts, T, min_tokens=4, min_step=32):
     """Experts of one step by the kernel that serves them: `counts` holds the
     pairs routed to each expert.  In steps of at least `min_step` tokens a
@@ -708,6 +822,8 @@ def main():
         run_batched(args)
     elif args.workload == "prefill":
         run_prefill(args)
+    elif args.workload == "storage":
+        run_storage(args)
     else:
         run_ours(args)
 

@@ -171,6 +171,13 @@ static int check_cfg(const MoeConfig* c) {
 
 extern "C" const char* moe_last_error(void) { return g_err.c_str(); }
 
+void moeq4_set_error(const char* msg) { g_err = msg; }
+
+// storage tier (store.cu)
+size_t moeq4_store_blob(const moe_store* st);
+int moeq4_store_fill(moe_store* st, int layer, const int32_t* experts, const int32_t* slot, int n,
+                     uint8_t* slots, cudaStream_t copy, cudaEvent_t copy_done);
+
 extern "C" size_t moe_blob_bytes(int hidden, int inter) {
     if (hidden <= 0 || inter <= 0 || hidden % MOE_GROUP || inter % MOE_GROUP) return 0;
     return BlobLayout(hidden, inter).bytes;
@@ -725,6 +732,19 @@ static int issue_fills(moe_ctx* c, const MoeLayer* L, cudaStream_t s, cudaStream
     if (nm < 0) return fail(MOE_ERR_CACHE_STATE, "LFU table is invalid (an earlier fill failed)");
     const uint8_t* store = static_cast<const uint8_t*>(L->host_store);
     uint8_t* slots = static_cast<uint8_t*>(L->slots);
+    if (L->store && !L->host_store) {
+        // storage tier: parallel pread into staging, then one copy per blob
+        std::vector<int32_t> ex(nm), sl(nm);
+        for (int i = 0; i < nm; i++) { ex[i] = c->miss_host[2 * i]; sl[i] = c->miss_host[2 * i + 1]; }
+        const int rc = moeq4_store_fill(const_cast<moe_store*>(L->store), L->store_layer, ex.data(), sl.data(),
+                                        nm, slots, cs, c->ev_copy);
+        if (rc != MOE_OK) {
+            k_lfu_invalidate<<<1, 1, 0, s>>>(L->lfu);
+            return rc;
+        }
+        CK(cudaStreamWaitEvent(s, c->ev_copy, 0));
+        return MOE_OK;
+    }
     for (int i = 0; i < nm; i++) {
         const int e = c->miss_host[2 * i], slot = c->miss_host[2 * i + 1];
         cudaError_t err = cudaSuccess;
@@ -875,6 +895,15 @@ static int layer_streaming_chunk(moe_ctx* c, const MoeLayer* L, __half* x, int T
                     static_cast<const uint8_t*>(dstore), slots, stride, c->plan_dev + (pairs - c->plan_host) + 2 * off[b],
                     c->plan_dev + 1 + (max_b + 1) + b, E, MOE_MAX_SLOTS);
                 CKL();
+            } else if (L->store && !L->host_store) {
+                std::vector<int32_t> ex(n), sl(n);
+                for (int m = 0; m < n; m++) { ex[m] = pairs[2 * (off[b] + m)]; sl[m] = pairs[2 * (off[b] + m) + 1]; }
+                const int rc = moeq4_store_fill(const_cast<moe_store*>(L->store), L->store_layer, ex.data(),
+                                                sl.data(), n, slots, cs, c->ev_copy);
+                if (rc != MOE_OK) {
+                    k_lfu_invalidate<<<1, 1, 0, s>>>(L->lfu);
+                    return rc;
+                }
             } else {
                 for (int m = off[b]; m < off[b + 1]; m++) {
                     const int e = pairs[2 * m], sl = pairs[2 * m + 1];
@@ -963,12 +992,16 @@ extern "C" int moe_layer_decode(moe_ctx* c, const MoeLayer* L, moe_half* x, int 
         if (!aligned16(L->experts)) return fail(MOE_ERR_ALIGNMENT, "experts must be 16-byte aligned");
         return layer_resident(c, L, reinterpret_cast<__half*>(x), T, o, flags, main);
     }
-    if (!L->host_store || !L->slots || !L->lfu || !copy)
-        return fail(MOE_ERR_INVALID_ARG, "streaming mode needs host_store, slots, lfu and a copy stream");
+    if ((!L->host_store && !L->store) || !L->slots || !L->lfu || !copy)
+        return fail(MOE_ERR_INVALID_ARG, "streaming mode needs host_store or store, slots, lfu and a copy stream");
+    if (L->store && !L->host_store && (flags & MOE_DEVICE_FILL))
+        return fail(MOE_ERR_INVALID_ARG, "MOE_DEVICE_FILL reads host_store; a store is read by the host");
+    if (L->store && !L->host_store && moeq4_store_blob(L->store) != BlobLayout(c->cfg.hidden, c->cfg.inter).bytes)
+        return fail(MOE_ERR_INVALID_ARG, "the store's blob size does not match the layer shape");
     if (T > 1 && !c->grouped_ok)
         return fail(MOE_ERR_UNSUPPORTED_SHAPE, "streaming chunks need the grouped kernels, whose tiles "
                     "do not fit this shape");
-    if (!aligned16(L->slots) || !aligned16(L->lfu) || !aligned16(L->host_store))
+    if (!aligned16(L->slots) || !aligned16(L->lfu) || (L->host_store && !aligned16(L->host_store)))
         return fail(MOE_ERR_ALIGNMENT, "moe_layer_decode: pointers must be 16-byte aligned");
     if (T > 1) return layer_streaming_chunk(c, L, reinterpret_cast<__half*>(x), T, o, flags, main, copy);
     return layer_streaming(c, L, reinterpret_cast<__half*>(x), o, flags, main, copy);

@@ -32,7 +32,9 @@ EXPORTS = ("moe_ctx_create", "moe_ctx_destroy", "moe_ctx_check", "moe_ctx_trace"
            "moe_last_error", "moe_blob_bytes",
            "moe_router_topk", "moe_expert_ffn_q4", "moe_combine", "moe_lfu_init",
            "moe_cache_lookup_lfu", "moe_layer_decode", "moe_stack_decode",
-           "moe_router_topk_noalloc", "moe_set_mma_min_tokens", "moe_set_wait_ns")
+           "moe_router_topk_noalloc", "moe_set_mma_min_tokens", "moe_set_wait_ns",
+           "moe_store_stride", "moe_store_open", "moe_store_close", "moe_store_read",
+           "moe_store_stats")
 
 
 class MoeError(RuntimeError):
@@ -52,7 +54,8 @@ class CMoeConfig(ctypes.Structure):
 class CMoeLayer(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "router_w", "router_scale", "router_bias", "shared_blob", "experts",
-        "host_store", "slots", "lfu")]
+        "host_store", "slots", "lfu", "store")] + [
+        ("store_layer", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class CMoeLayerOut(ctypes.Structure):
@@ -104,6 +107,12 @@ def load() -> ctypes.CDLL:
                               ctypes.POINTER(CMoeLayerOut), i32, P, P], i32),
         "moe_stack_decode": ([P, P, i32, P, i32, P, P], i32),
         "moe_router_topk_noalloc": ([i32, i32, i32, i32, P, P, P, P, i32, P, P, P], i32),
+        "moe_store_stride": ([ctypes.c_size_t], ctypes.c_size_t),
+        "moe_store_open": ([ctypes.c_char_p, i32, i32, ctypes.c_size_t, i32, i32, ctypes.POINTER(P)], i32),
+        "moe_store_close": ([P], i32),
+        "moe_store_read": ([P, i32, P, i32, P], i32),
+        "moe_store_stats": ([P, ctypes.POINTER(ctypes.c_ulonglong), ctypes.POINTER(ctypes.c_double),
+                             ctypes.POINTER(ctypes.c_int)], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -263,10 +272,12 @@ class Layer:
     """A layer's buffers (torch tensors) as the C MoeLayer struct."""
 
     def __init__(self, router_w, router_scale, router_bias=None, shared=None, experts=None,
-                 host_store=None, slots=None, lfu=None):
-        self.keep = (router_w, router_scale, router_bias, shared, experts, host_store, slots, lfu)
+                 host_store=None, slots=None, lfu=None, store=None, store_layer=0):
+        self.keep = (router_w, router_scale, router_bias, shared, experts, host_store, slots, lfu,
+                     store)
         self.c = CMoeLayer(_ptr(router_w), _ptr(router_scale), _ptr(router_bias), _ptr(shared),
-                           _ptr(experts), _ptr(host_store), _ptr(slots), _ptr(lfu))
+                           _ptr(experts), _ptr(host_store), _ptr(slots), _ptr(lfu),
+                           None if store is None else store.handle, int(store_layer), 0)
 
     @classmethod
     def from_dict(cls, d, **kw):
@@ -286,3 +297,58 @@ def moe_stack_decode(ctx, layers, h, T, y_last=None, stream=None):
     arr = (CMoeLayer * len(layers))(*[l.c for l in layers])
     _check(load().moe_stack_decode(ctx.handle, ctypes.cast(arr, ctypes.c_void_p), len(layers),
                                    _ptr(h), T, _ptr(y_last), _stream(stream)))
+
+
+def store_stride(blob_bytes: int) -> int:
+    """moe_store_stride: bytes per blob in an expert file (padded to 4 KiB)."""
+    return int(load().moe_store_stride(int(blob_bytes)))
+
+
+class Store:
+    """moe_store_open / moe_store_close: an expert file read with parallel pread."""
+
+    def __init__(self, path, n_layers, n_experts, blob_bytes, n_threads=8, n_staging=16):
+        h = ctypes.c_void_p()
+        _check(load().moe_store_open(str(path).encode(), n_layers, n_experts, blob_bytes, n_threads,
+                                     n_staging, ctypes.byref(h)))
+        self.handle = h.value
+        self.blob_bytes = blob_bytes
+
+    def read(self, layer, experts, dst):
+        """moe_store_read into the host arrays dst[i] (numpy uint8, blob_bytes each)."""
+        import numpy as np
+        ex = np.ascontiguousarray(np.asarray(experts, np.int32))
+        ptrs = (ctypes.c_void_p * len(dst))(*[d.ctypes.data for d in dst])
+        _check(load().moe_store_read(self.handle, int(layer), ex.ctypes.data, len(ex),
+                                     ctypes.cast(ptrs, ctypes.c_void_p)))
+
+    def stats(self):
+        """moe_store_stats: (bytes read, seconds reading, O_DIRECT in use)."""
+        b, t, d = ctypes.c_ulonglong(), ctypes.c_double(), ctypes.c_int()
+        _check(load().moe_store_stats(self.handle, ctypes.byref(b), ctypes.byref(t), ctypes.byref(d)))
+        return int(b.value), float(t.value), bool(d.value)
+
+    def close(self):
+        if self.handle:
+            load().moe_store_close(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def write_expert_file(path, layers_experts, blob_bytes):
+    """Writes an expert file in the store's format: for each layer (a uint8
+    array or tensor [E][blob_bytes]) each blob padded to store_stride bytes."""
+    import numpy as np
+    stride = store_stride(blob_bytes)
+    pad = np.zeros(stride - blob_bytes, np.uint8)
+    with open(path, "wb") as f:
+        for ex in layers_experts:
+            a = ex.cpu().numpy() if hasattr(ex, "cpu") else np.asarray(ex)
+            for e in range(a.shape[0]):
+                f.write(a[e].tobytes())
+                f.write(pad.tobytes())

@@ -354,6 +354,8 @@ int moe_cache_lookup_lfu(moe_ctx *ctx, MoeLfuTable *table,
  */
 enum { MOE_PRENORM = 1, MOE_DEVICE_FILL = 2 };
 
+typedef struct moe_store moe_store;    /* expert file reader (below) */
+
 typedef struct {
     const int8_t *router_w;       /* device int8 [E][H] */
     const moe_half *router_scale; /* device fp16 [E] */
@@ -363,6 +365,10 @@ typedef struct {
     const void *host_store;       /* streaming: pinned host [E] blobs */
     void *slots;                  /* streaming: device [n_slots] blobs */
     MoeLfuTable *lfu;             /* streaming: device table */
+    const moe_store *store;       /* streaming without host_store: misses read
+                                     from this expert file (storage tier) */
+    int32_t store_layer;          /* the layer's index in the store */
+    int32_t reserved;             /* zero */
 } MoeLayer;
 
 typedef struct {
@@ -376,6 +382,49 @@ typedef struct {
 int moe_layer_decode(moe_ctx *ctx, const MoeLayer *layer, moe_half *x, int T,
                      const MoeLayerOut *out, int flags, moe_stream_t main,
                      moe_stream_t copy);
+
+/* ------------------------------------------------------- expert store ----
+ * The storage tier of the cache ([DS] "Trois optimisations clés" items 2-3:
+ * experts streamed from the SSD and read ahead with parallel pread; [LH] 04
+ * "Le pipeline de traitement" steps 3-4: only the missing experts are read).
+ *
+ * File format: n_layers x n_experts expert blobs (each moe_blob_bytes of the
+ * layer shape), layer-major; each blob is padded to moe_store_stride(blob)
+ * bytes (the next multiple of 4096), so blob (l, e) starts at byte
+ * (l * n_experts + e) * stride.  The padding keeps every read aligned to 4
+ * KiB, so the store opens the file with O_DIRECT (no page cache) where the
+ * file system accepts it, else with buffered reads.
+ *
+ * A streaming MoeLayer with host_store == NULL and store set reads its misses
+ * from the file: after the cache lookup the host reads the missing blobs with
+ * n_threads threads (each pread of at most 1 MiB) into the store's pinned
+ * staging buffers (n_staging blobs, allocated by moe_store_open; page-aligned
+ * host memory when no GPU is present), then copies each into its slot on the
+ * copy stream, while the shared expert computes.  MOE_DEVICE_FILL is refused
+ * with a store (the device cannot read the file).  A failed read marks the
+ * table invalid and returns MOE_ERR_CACHE_STATE.  One store serves one
+ * caller thread at a time. */
+size_t moe_store_stride(size_t blob_bytes);
+
+/* Opens path for n_layers x n_experts blobs of blob_bytes (a multiple of 16);
+ * starts n_threads reader threads (1..256) and allocates n_staging staging
+ * blobs (1..4096).  MOE_ERR_INVALID_ARG when the file is missing or shorter
+ * than the format needs; the caller closes the store. */
+int moe_store_open(const char *path, int n_layers, int n_experts, size_t blob_bytes,
+                   int n_threads, int n_staging, moe_store **out);
+
+/* Stops the threads, closes the file and frees the staging.  NULL accepted. */
+int moe_store_close(moe_store *store);
+
+/* Reads blobs (layer, experts[i]) for i < n into host buffers dst[i] (any
+ * host memory, blob_bytes each), n_staging at a time in parallel. */
+int moe_store_read(moe_store *store, int layer, const int32_t *experts, int n,
+                   void *const *dst);
+
+/* Totals since open: bytes of blobs read, seconds spent reading (wall
+ * clock of the read calls), and whether reads bypass the page cache. */
+int moe_store_stats(const moe_store *store, unsigned long long *bytes,
+                    double *seconds, int *direct);
 
 /* ------------------------------------------------------------- stack ----
  * Decodes T tokens one after another through n_layers resident layers
