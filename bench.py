@@ -291,9 +291,11 @@ def run_ours(args):
 # source reports null (the counters describe a different kernel).
 KERNEL_SRC = os.path.join(ROOT, "bit_quantized_expert_int8_b200", "csrc", "layer_fused.cuh")
 TRAFFIC_BY_SOURCE = {
-    # ncu --set full, one launch of the 30-layer bench layers (hidden 2816,
-    # top-8): dram__bytes_read.sum 37,284,864 + dram__bytes_write.sum 43,008
+    # ncu --set full, one launch of the bench layers (hidden 2816, top-8),
+    # 16-bit x digits: dram__bytes_read.sum 37,284,864 + write 43,008
     "ab523b1bf6c48f302f20a8d0fa33bdea867f6816a4e0a6fbc4a69b12422ad079": 37327872,
+    # the same capture with 24-bit x digits: read 37,290,496 + write 114,432
+    "c31f5378bd41ff1c3afc7da62ad3dfbbf79f3cba4022471fda56907f7fdcafba": 37404928,
 }
 
 
