@@ -104,3 +104,45 @@ def test_gateup_fold_matches_oracle():
     h = np.array([oracle.gelu(g_) for g_ in gate]) * up
     rel = np.linalg.norm(h - h_ref) / np.linalg.norm(h_ref)
     assert rel < 1e-5, rel
+
+
+def test_fp16_dequantised_weights_would_miss_the_absolute_bound():
+    """Why the tensor-core kernels keep the codes exact and fold scale and
+    bias per group: a design that dequantises each weight once to fp16 (one
+    rounding of s q + b, then one accumulator over all of K) keeps rel L2
+    near 2e-4 but misses the 2e-3 absolute bound on heavy-tailed rows
+    through the shared expert (|y| near 10), while the exact codes meet it."""
+    H, I, T = 2816, 2112, 4
+    seed = 200 + I
+    w_gu = synth.randn((2 * I, H), seed, "cpu", synth.WEIGHT_STD)
+    w_dn = synth.randn((H, I), seed + 1, "cpu", synth.WEIGHT_STD)
+    qg_w, sg, bg = synth.quantize_q4(w_gu)
+    qd_w, sd, bd = synth.quantize_q4(w_dn)
+    blob = synth.pack_blob(qg_w, sg, bg, qd_w, sd, bd, H, I).numpy()
+    xd = synth.student_t_tokens(T, H, seed=seed + 2).double().numpy()
+    qg, qd = _unpack(qg_w), _unpack(qd_w)
+
+    def ffn(wg, wd):
+        gu = xd @ wg.T
+        g, u = gu[:, :I], gu[:, I:]
+        h = np.vectorize(lambda v: oracle.gelu(v, 0))(g) * u
+        return h @ wd.T
+
+    def exact(q, s, b):
+        R, K = q.shape
+        return (q.reshape(R, K // G, G) * s[..., None] + b[..., None]).reshape(R, K)
+
+    def f16(q, s, b):
+        return exact(q, s, b).astype(np.float16).astype(np.float64)
+
+    s_g, b_g, s_d, b_d = (t.double().numpy() for t in (sg, bg, sd, bd))
+    y16 = ffn(f16(qg, s_g, b_g), f16(qd, s_d, b_d))
+    yex = ffn(exact(qg, s_g, b_g), exact(qd, s_d, b_d))
+    worst16 = worst_ex = 0.0
+    for t in range(T):
+        ref, _ = oracle.expert_ffn(blob, H, I, xd[t])
+        assert np.linalg.norm(y16[t] - ref) / np.linalg.norm(ref) < 1e-3
+        worst16 = max(worst16, np.abs(y16[t] - ref).max())
+        worst_ex = max(worst_ex, np.abs(yex[t] - ref).max())
+    assert worst16 > 2e-3          # single fp16 weights: over the absolute bound
+    assert worst_ex < 1e-9         # exact weights (the kernels' codes + fold): at rounding level
