@@ -167,8 +167,12 @@ __device__ __forceinline__ bool fused_aborted(const int* status) {
     return ld_relaxed_s32(status) != 0;
 }
 
-// Wait on an mbarrier phase, bounded in time; gives up early when another
-// thread has already recorded a failure.
+// Waits longer than this look at the status word in global memory (a load
+// that can take microseconds under load, so ordinary waits never issue it).
+constexpr unsigned long long kAbortCheckNs = 20000;
+
+// Wait on an mbarrier phase, bounded in time; once the wait is long, gives up
+// early when another thread has already recorded a failure.
 __device__ __forceinline__ bool fused_wait_bar(uint64_t* bar, uint32_t parity, int* status,
                                                unsigned long long bound = kWaitNs) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -176,8 +180,9 @@ __device__ __forceinline__ bool fused_wait_bar(uint64_t* bar, uint32_t parity, i
     for (unsigned it = 1;; it++) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 31) == 0) {
-            if (fused_aborted(status)) return false;
-            if (gtimer_ns() - t0 > bound) { fused_fail(status); return false; }
+            const unsigned long long el = gtimer_ns() - t0;
+            if (el > bound) { fused_fail(status); return false; }
+            if (el > kAbortCheckNs && fused_aborted(status)) return false;
         }
     }
 }

@@ -116,9 +116,11 @@ struct moe_ctx {
     bool mma_ok = false;               // tensor-core kernels usable for this shape
     int mma_min_tok = 0;               // bucket size from which they run (0: never)
     __nv_bfloat16* h_pl = nullptr;     // [2][maxT * (k + 1)][maxI] h as bf16 hi / lo planes
-    float* h_sum = nullptr;            // [maxT * (k + 1)][maxI / 64] group sums of h
+    float* h_sum = nullptr;            // [maxT * (k + 1)][hsum_stride] group sums of h
+    int hsum_stride = 0;               // maxI / 64 rounded up to 4 floats (16-byte rows)
+    int xg_stride = 0;                 // H / 64 rounded up to 4 floats
     __half* xs = nullptr;              // [maxT * (k + 1)][H] x rows: tokens, then pairs by bucket
-    float* xg_sum = nullptr;           // [maxT * (k + 1)][H / 64] their group sums
+    float* xg_sum = nullptr;           // [maxT * (k + 1)][xg_stride] their group sums
     int* e_off = nullptr;              // [E + 1] pairs per expert (prefix)
     int* plist = nullptr;              // [maxT * k] pair indices grouped by expert
     uint32_t* dlimb = nullptr;         // packed intermediate of the fused kernel
@@ -219,26 +221,27 @@ static PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
 }
 
 // Tensor map over the codes of tiled expert blobs: dims {row bytes, rows per
-// tile, tiles, experts}; one copy takes 32 bytes of 128 rows (box_tiles tiles).
+// tile, tiles, experts}; one copy takes 64 bytes (128 columns) of 128 rows
+// (box_tiles tiles), 64-byte swizzle.
 static bool encode_codes(CUtensorMap* m, const void* base, int row_bytes, int rows_per_tile,
                          size_t tile_stride, int tiles, size_t expert_stride, int experts, int box_tiles) {
     const cuuint64_t dims[4] = {(cuuint64_t)row_bytes, (cuuint64_t)rows_per_tile, (cuuint64_t)tiles,
                                 (cuuint64_t)experts};
     const cuuint64_t strides[3] = {(cuuint64_t)row_bytes, (cuuint64_t)tile_stride, (cuuint64_t)expert_stride};
-    const cuuint32_t box[4] = {32u, (cuuint32_t)rows_per_tile, (cuuint32_t)box_tiles, 1u};
+    const cuuint32_t box[4] = {64u, (cuuint32_t)rows_per_tile, (cuuint32_t)box_tiles, 1u};
     const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
     return tmap_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box,
-                          es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Tensor map over 16-bit rows: dims {cols, rows, planes}; one copy takes
-// 64 columns x 64 rows of every plane, 128-byte swizzle.
+// 64 columns x box_rows rows of every plane, 128-byte swizzle.
 static bool encode_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int cols, int rows,
-                        int planes) {
+                        int planes, int box_rows) {
     const cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)planes};
     const cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)cols * 2 * rows};
-    const cuuint32_t box[3] = {64u, 64u, (cuuint32_t)planes};
+    const cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, (cuuint32_t)planes};
     const cuuint32_t es[3] = {1u, 1u, 1u};
     return tmap_encoder()(m, dt, 3, const_cast<void*>(base), dims, strides, box, es,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -263,18 +266,15 @@ static cudaError_t setup_grouped(moe_ctx* c) {
     if (e == cudaSuccess)
         e = raise_smem(k_down_grouped<true>, (int)dn);
     if (e != cudaSuccess) return e;
-    // tensor-core kernels: 4 gate/up tiles (64 indices) or 128 down rows per CTA
-    const size_t tc_gu = tc_smem_bytes<false>(g.hidden), tc_dn = tc_smem_bytes<true>(c->maxI);
+    // tensor-core kernels: items of 4 gate/up tiles (64 indices) or 128 down rows
+    const size_t tc_gu = tc_smem_bytes<false>(g.hidden, c->xg_stride);
+    const size_t tc_dn = tc_smem_bytes<true>(c->maxI, c->hsum_stride);
     if (!tmap_encoder() || tc_gu > (size_t)optin || tc_dn > (size_t)optin || g.hidden % kMmaRows ||
         g.inter % 64 || g.inter_shared % 64)
         return cudaSuccess;
-    e = raise_smem(k_ffn_tc<false, false>, (size_t)tc_gu);
+    e = raise_smem(k_ffn_tc<false>, (size_t)tc_gu);
     if (e == cudaSuccess)
-        e = raise_smem(k_ffn_tc<false, true>, (size_t)tc_gu);
-    if (e == cudaSuccess)
-        e = raise_smem(k_ffn_tc<true, false>, (size_t)tc_dn);
-    if (e == cudaSuccess)
-        e = raise_smem(k_ffn_tc<true, true>, (size_t)tc_dn);
+        e = raise_smem(k_ffn_tc<true>, (size_t)tc_dn);
     if (e != cudaSuccess) return e;
     c->mma_ok = true;
     c->mma_min_tok = kMmaDefaultMinTokens;
@@ -366,8 +366,10 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     size_t o_plist = take(T * k * sizeof(int));
     size_t o_hpl = take(2 * P * (size_t)c->maxI * sizeof(__nv_bfloat16));   // h hi / lo planes
     size_t o_xs = take(P * H * sizeof(__half));                              // x rows, bucket order
-    size_t o_xgsum = take(P * (H / 64) * sizeof(float));                     // their group sums
-    size_t o_hsum = take(P * (size_t)(c->maxI / 64) * sizeof(float));        // h group sums
+    c->xg_stride = (int)((H / 64 + 3) / 4 * 4);
+    c->hsum_stride = (c->maxI / 64 + 3) / 4 * 4;
+    size_t o_xgsum = take(P * (size_t)c->xg_stride * sizeof(float));         // their group sums
+    size_t o_hsum = take(P * (size_t)c->hsum_stride * sizeof(float));        // h group sums
     int n_sms_dev = 0;
     cudaDeviceGetAttribute(&n_sms_dev, cudaDevAttrMultiProcessorCount, c->device);
     size_t o_trace = take((size_t)(n_sms_dev > 0 ? n_sms_dev : 1) * kTraceWords * sizeof(unsigned long long));
@@ -642,75 +644,68 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
         const bool tc = tau > 0 && T >= kMmaMinStep;
         const bool tc_shared = tc && T >= tau;
         const int cap = tc ? tau : 0x7fffffff;
-        const int tiles = (T + kMmaTok - 1) / kMmaTok;
         const int P = T * (k + 1), hs = c->maxI;
         __nv_bfloat16 *hh = c->h_pl, *hl = c->h_pl + (size_t)P * hs;
         k_group_pairs<<<1, 1024, 0, s>>>(idx, T * k, E, c->e_off, c->plist);
         CKL();
-        CUtensorMap m_cgr, m_cgs, m_cdr, m_cds, m_x, m_h;
+        CUtensorMap m_cgr, m_cgs, m_cdr, m_cds, m_x[3], m_h[3];
         TcArgs ta{};
         if (tc) {
             // x rows in bucket order (tokens first) with their group sums; this call's tensor maps
             k_gather_x<<<dim3((H + 2047) / 2048, P < 65535 ? P : 65535), 256, 0, s>>>(
-                xin, H, T, k, P, c->plist, c->xs, c->xg_sum);
+                xin, H, T, k, P, c->plist, c->xs, c->xg_sum, c->xg_stride);
             CKL();
             const BlobLayout Lr(H, I), Ls(H, Is);
             const size_t sb = Ls.bytes;
-            if (!encode_codes(&m_cgr, ex, H / 2, 32, Lr.gu_tile, I / 16, stride, E, 4) ||
-                !encode_codes(&m_cgs, sh, H / 2, 32, Ls.gu_tile, Is / 16, sb, 1, 4) ||
-                !encode_codes(&m_cdr, ex + Lr.dn_base, I / 2, 16, Lr.dn_tile, H / 16, stride, E, 8) ||
-                !encode_codes(&m_cds, sh + Ls.dn_base, Is / 2, 16, Ls.dn_tile, H / 16, sb, 1, 8) ||
-                !encode_rows(&m_x, c->xs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, H, P, 1) ||
-                !encode_rows(&m_h, hh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hs, P, 2))
-                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-            ta.H = H; ta.T = T; ta.k = k; ta.min_tok = tau; ta.gelu = g.gelu;
+            bool enc = encode_codes(&m_cgr, ex, H / 2, 32, Lr.gu_tile, I / 16, stride, E, 4) &&
+                       encode_codes(&m_cgs, sh, H / 2, 32, Ls.gu_tile, Is / 16, sb, 1, 4) &&
+                       encode_codes(&m_cdr, ex + Lr.dn_base, I / 2, 16, Lr.dn_tile, H / 16, stride, E, 8) &&
+                       encode_codes(&m_cds, sh + Ls.dn_base, Is / 2, 16, Ls.dn_tile, H / 16, sb, 1, 8);
+            for (int b = 0; b < 3 && enc; b++)
+                enc = encode_rows(&m_x[b], c->xs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, H, P, 1, 16 << b) &&
+                      encode_rows(&m_h[b], hh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hs, P, 2, 16 << b);
+            if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+            ta.H = H; ta.T = T; ta.k = k; ta.E = E; ta.gelu = g.gelu;
+            ta.Ir = I; ta.Is = Is; ta.min_tok = tau; ta.do_shared = tc_shared ? 1 : 0;
             ta.e_off = c->e_off; ta.list = c->plist;
-            ta.h_hi = hh; ta.h_lo = hl; ta.h_sum = c->h_sum; ta.hs = hs;
+            ta.h_hi = hh; ta.h_lo = hl; ta.h_sum = c->h_sum; ta.hs = hs; ta.hsum_stride = c->hsum_stride;
             ta.y_pairs = c->y_pairs; ta.status = c->status;
         }
         const int chunks = (T + kGrpChunk - 1) / kGrpChunk;
         k_gateup_grouped<false><<<dim3(I / 16, E), kGrpThreads, grouped_smem_gu(H), s>>>(
             ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
         CKL();
-        TcArgs gu = ta;
-        gu.b_sum = c->xg_sum;
-        gu.bs_stride = H / 64;
-        if (tc) {
-            gu.Ie = I;
-            k_ffn_tc<false, false><<<dim3(I / 64, E, tiles), kTcThreads, tc_smem_bytes<false>(H), s>>>(
-                m_cgr, m_x, ex, stride, sh, gu);
-            CKL();
-        }
-        if (tc_shared) {
-            gu.Ie = Is;
-            k_ffn_tc<false, true><<<dim3(Is / 64, 1, tiles), kTcThreads, tc_smem_bytes<false>(H), s>>>(
-                m_cgs, m_x, ex, stride, sh, gu);
-        } else {
+        if (!tc_shared) {
             k_gateup_grouped<true><<<dim3(Is / 16, 1, chunks), kGrpThreads, grouped_smem_gu(H), s>>>(
                 ex, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
+            CKL();
         }
-        CKL();
+        if (tc) {
+            TcArgs gu = ta;
+            gu.b_sum = c->xg_sum;
+            gu.bs_stride = c->xg_stride;
+            gu.kmax = H;
+            k_ffn_tc<false><<<c->n_sms, kTcThreads, tc_smem_bytes<false>(H, c->xg_stride), s>>>(
+                m_cgr, m_cgs, m_x[0], m_x[1], m_x[2], ex, stride, sh, gu);
+            CKL();
+        }
         k_down_grouped<false><<<dim3(H / 16, E), kGrpThreads, grouped_smem_dn(I), s>>>(
             ex, stride, sh, H, I, T, c->e_off, c->plist, cap, c->h_ws, c->maxI, c->y_pairs);
         CKL();
-        TcArgs dn = ta;
-        dn.b_sum = c->h_sum;
-        dn.bs_stride = hs / 64;
-        if (tc) {
-            dn.Ie = I;
-            k_ffn_tc<true, false><<<dim3(H / kMmaRows, E, tiles), kTcThreads, tc_smem_bytes<true>(I), s>>>(
-                m_cdr, m_h, ex, stride, sh, dn);
-            CKL();
-        }
-        if (tc_shared) {
-            dn.Ie = Is;
-            k_ffn_tc<true, true><<<dim3(H / kMmaRows, 1, tiles), kTcThreads, tc_smem_bytes<true>(Is), s>>>(
-                m_cds, m_h, ex, stride, sh, dn);
-        } else {
+        if (!tc_shared) {
             k_down_grouped<true><<<dim3(H / 16, 1, chunks), kGrpThreads, grouped_smem_dn(Is), s>>>(
                 ex, stride, sh, H, Is, T, c->e_off, c->plist, cap, c->h_ws, c->maxI, c->y_pairs);
+            CKL();
         }
-        CKL();
+        if (tc) {
+            TcArgs dn = ta;
+            dn.b_sum = c->h_sum;
+            dn.bs_stride = c->hsum_stride;
+            dn.kmax = c->maxI;
+            k_ffn_tc<true><<<c->n_sms, kTcThreads, tc_smem_bytes<true>(c->maxI, c->hsum_stride), s>>>(
+                m_cdr, m_cds, m_h[0], m_h[1], m_h[2], ex, stride, sh, dn);
+            CKL();
+        }
     } else {
         k_build_pairs<<<(P + 127) / 128, 128, 0, s>>>(L->shared_blob, g.inter_shared,
                                                       static_cast<const uint8_t*>(L->experts), stride,
