@@ -722,7 +722,7 @@ def run_storage(args):
         os.unlink(path)
 
 
-def bucket_split(counts, T, min_tokens=4, min_step=32):
+def bucket_split(counts, T, min_tokens=1, min_step=32):
     """Experts of one step by the kernel that serves them: `counts` holds the
     pairs routed to each expert.  In steps of at least `min_step` tokens a
     bucket of `min_tokens` or more pairs runs on tcgen05; every other used
@@ -788,8 +788,7 @@ def run_batched(args):
         if T == 1:
             path = "fused single-token kernel"
         elif T >= 32:
-            path = ("tcgen05 kernels (shared expert, buckets of >= 4 pairs) + CUDA-core grouped "
-                    "kernels (smaller buckets)")
+            path = "tcgen05 kernels (shared expert and every routed bucket, one persistent launch per FFN half)"
         else:
             path = "CUDA-core grouped kernels"
         lines.append({"tokens": T, "us_per_step": round(us, 2),
@@ -811,7 +810,7 @@ def run_batched(args):
     print(json.dumps({"metric": METRIC, "workload": "batched sweep, one layer", "unit": UNIT,
                       "timing": f"median of {REPEATS} runs of each step size", "clocks": clk,
                       "peak_gbs": hbm, "peak_kind": kind, "tensor_peak_tflops": tpk,
-                      "tensor_peak_kind": tkind, "mma_min_tokens": 4, "sweep": lines}), flush=True)
+                      "tensor_peak_kind": tkind, "mma_min_tokens": 1, "sweep": lines}), flush=True)
 
 
 def main():

@@ -33,8 +33,8 @@
 //                64-column halves, 128-byte swizzle; down: both planes) sized
 //                to the tile (16, 32 or 64 rows);
 //   warp 1       MMA issuer: per stage 4 (down: 8) MMAs per group with A in
-//                tensor memory, then one commit that frees the ring slot and
-//                the A buffer and publishes the accumulator;
+//                tensor memory, then one commit that publishes the stage's
+//                accumulators and frees its ring slot and A buffer;
 //   warps 2..5   converters: codes -> 16-bit A straight into tensor memory
 //                (tcgen05.st, one row per thread), so A costs no shared-
 //                memory bandwidth;
@@ -59,7 +59,7 @@ namespace moeq4 {
 
 constexpr int kMmaRows = 128;                          // M: weight rows per item (TMEM lanes)
 constexpr int kMmaTok = 64;                            // tokens per item at most (N: rounded up to 16)
-constexpr int kMmaDefaultMinTokens = 4;                // bucket size from which a routed expert runs here
+constexpr int kMmaDefaultMinTokens = 1;                // bucket size from which a routed expert runs here
 constexpr int kMmaMinStep = 32;                        // tokens in a step before any expert runs here
 constexpr int kTcStageK = 128;                         // K per pipeline stage: two scale groups
 constexpr int kTcCodeBytes = kMmaRows * kTcStageK / 2; // codes of one stage (8 KB)
@@ -365,7 +365,6 @@ struct TcFold {
     uint32_t g;              // stages consumed so far
     int m, q4, half, lane, tid;
     uint32_t t_acc0;         // TMEM address of this lane quarter's accumulators
-    uint64_t* stage_done;
     uint64_t* acc_empty;
     uint64_t* acc_full;
     TcAccRing ring;
@@ -404,6 +403,70 @@ __device__ __forceinline__ int tc_fold_item(TcFold& f, const TcItem& d, int j, c
 #pragma unroll
     for (int q = 0; q < CW; q++) acc[q] = 0.f;
     const uint32_t t_acc = f.t_acc0 + (uint32_t)c0;
+    if (CW == 8) {
+        // 8 columns: up to 2 stages per TMEM load batch (one wait on the last
+        // stage's commit, which follows every earlier MMA)
+        constexpr int NB = 2;
+        for (int c = 0; c < d.nst;) {
+            const int nb = min(NB, d.nst - c);
+            uint32_t acol[NB];
+#pragma unroll
+            for (int b = 0; b < NB; b++) acol[b] = b < nb ? f.ring.take(2 * gst) : 0u;
+            const uint32_t gl = g + (uint32_t)nb - 1;
+            if (!fused_wait_bar(&f.acc_full[gl % kTcAcc], (gl / kTcAcc) & 1u, f.status)) return -1;
+            tc_fence_after();
+            uint32_t P[NB][2][8];
+            if (on) {
+#pragma unroll
+                for (int b = 0; b < NB; b++) {
+                    if (b < nb) {
+                        tmem_ld8_nw(t_acc + acol[b], P[b][0]);
+                        if (d.ng - 2 * (c + b) > 1) tmem_ld8_nw(t_acc + acol[b] + gst, P[b][1]);
+                    }
+                }
+                tmem_ld_wait();
+            }
+            tc_fence_before();                        // the accumulators are free once in registers
+            __syncwarp();
+            if (f.lane == 0) {
+                for (int b = 0; b < nb; b++) mbar_arrive(&f.acc_empty[(g + b) % kTcAcc]);
+            }
+            if (on) {
+#pragma unroll
+                for (int b = 0; b < NB; b++) {
+                    if (b < nb) {
+                        const int G = 2 * (c + b);
+                        if (d.ng - G > 1) {
+                            float s0, s1, b0, b1;
+                            if (pair_sc) {
+                                const float2 sc2 = __half22float2(*reinterpret_cast<const __half2*>(scp + G));
+                                const float2 bi2 = __half22float2(*reinterpret_cast<const __half2*>(bip + G));
+                                s0 = sc2.x; s1 = sc2.y; b0 = bi2.x; b1 = bi2.y;
+                            } else {
+                                s0 = __half2float(scp[G]); s1 = __half2float(scp[G + 1]);
+                                b0 = __half2float(bip[G]); b1 = __half2float(bip[G + 1]);
+                            }
+#pragma unroll
+                            for (int q = 0; q < 8; q++) {
+                                const float2 S2 = *reinterpret_cast<const float2*>(gsp + q * bs + G);
+                                float v = fmaf(b0, S2.x, acc[q]);
+                                v = fmaf(s0, __uint_as_float(P[b][0][q]), v);
+                                v = fmaf(b1, S2.y, v);
+                                acc[q] = fmaf(s1, __uint_as_float(P[b][1][q]), v);
+                            }
+                        } else {
+                            const float s0 = __half2float(scp[G]), b0 = __half2float(bip[G]);
+#pragma unroll
+                            for (int q = 0; q < 8; q++)
+                                acc[q] = fmaf(s0, __uint_as_float(P[b][0][q]), fmaf(b0, gsp[q * bs + G], acc[q]));
+                        }
+                    }
+                }
+            }
+            c += nb;
+            g += (uint32_t)nb;
+        }
+    } else {
     for (int c = 0; c < d.nst; c++, g++) {
         const uint32_t ab = g % kTcAcc;
         const uint32_t acol = f.ring.take(2 * gst);
@@ -463,6 +526,7 @@ __device__ __forceinline__ int tc_fold_item(TcFold& f, const TcItem& d, int j, c
                 }
             }
         }
+    }
     }
     if (!DOWN) {
         // lanes < 16 hold gate rows, lanes >= 16 the up rows of the same 16
@@ -542,7 +606,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_cr, const __grid_constant__ CUte
     using S = TcShape<DOWN>;
     constexpr int R = S::kRing;
     extern __shared__ uint8_t tsm_raw[];
-    __shared__ __align__(8) uint64_t full_slot[R], stage_done[R], a_full[R];
+    __shared__ __align__(8) uint64_t full_slot[R], a_full[R];
     __shared__ __align__(8) uint64_t acc_empty[kTcAcc], acc_full[kTcAcc], ib_full[kTcItemBufs], ib_empty[kTcItemBufs];
     __shared__ __align__(8) uint64_t red_full[2];
     __shared__ uint32_t s_tmem;
@@ -598,7 +662,6 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_cr, const __grid_constant__ CUte
     if (tid == 0) {
         for (int i = 0; i < R; i++) {
             mbar_init(&full_slot[i], 1);
-            mbar_init(&stage_done[i], 1);                 // the MMA commit
             mbar_init(&a_full[i], 4);                     // converter warps
         }
         for (int i = 0; i < kTcAcc; i++) {
@@ -661,7 +724,12 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_cr, const __grid_constant__ CUte
                 const CUtensorMap* mc = d.shared ? &tm_cs : &tm_cr;
                 for (int c = 0; c < d.nst; c++, g++) {
                     const uint32_t slot = g % R;
-                    if (!fused_wait_bar(&stage_done[slot], ((g / R) & 1u) ^ 1u, status)) { ok = false; break; }
+                    // the slot's previous stage (g - R) has completed its MMAs
+                    if (g >= (uint32_t)R &&
+                        !fused_wait_bar(&acc_full[(g - R) % kTcAcc], ((g - R) / kTcAcc) & 1u, status)) {
+                        ok = false;
+                        break;
+                    }
                     const uint32_t sl = s_ring + slot * S::kSlot;
                     mbar_arrive_expect_tx(&full_slot[slot], kTcCodeBytes + 2u * bbytes);
                     tma_load_4d(sl, mc, 64 * c, 0, (DOWN ? 8 : 4) * d.sb, d.shared ? 0 : d.e, &full_slot[slot]);
@@ -715,13 +783,11 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_cr, const __grid_constant__ CUte
                                 tc_mma_ts(dacc, at, tc_sdesc_sw128(bt + brows * 128 + 32u * kk), idesc, 1u);
                         }
                     }
-                    mma_commit(&stage_done[slot]);
                     mma_commit(&acc_full[g % kTcAcc]);
                 }
             }
             // every commit has arrived before the CTA ends
             if (g > 0) {
-                mma_drain_wait(&stage_done[(g - 1) % R], ((g - 1) / R) & 1u);
                 mma_drain_wait(&acc_full[(g - 1) % kTcAcc], ((g - 1) / kTcAcc) & 1u);
             }
         }
@@ -736,7 +802,8 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_cr, const __grid_constant__ CUte
             for (int c = 0; c < d.nst; c++, g++) {
                 const uint32_t slot = g % R;
                 if (!fused_wait_bar(&full_slot[slot], (g / R) & 1u, status) ||
-                    !fused_wait_bar(&stage_done[slot], ((g / R) & 1u) ^ 1u, status)) {
+                    (g >= (uint32_t)R &&
+                     !fused_wait_bar(&acc_full[(g - R) % kTcAcc], ((g - R) / kTcAcc) & 1u, status))) {
                     ok = false;
                     break;
                 }
@@ -773,7 +840,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_cr, const __grid_constant__ CUte
         const uint32_t t_acc0 = tmem + ((uint32_t)(32 * q4) << 16) + kTcAccCol;
         TcFold f;
         f.a = &a; f.status = status; f.g = 0; f.m = m; f.q4 = q4; f.half = half; f.lane = lane;
-        f.tid = tid; f.t_acc0 = t_acc0; f.stage_done = stage_done; f.acc_empty = acc_empty;
+        f.tid = tid; f.t_acc0 = t_acc0; f.acc_empty = acc_empty;
         f.acc_full = acc_full;
         f.red_full = red_full; f.s_red = s_red;
         int j = 0;

@@ -114,6 +114,7 @@ struct moe_ctx {
     bool fused_ok = false;
     bool grouped_ok = false;           // multi-token steps grouped by expert
     bool mma_ok = false;               // tensor-core kernels usable for this shape
+    bool router_batch_ok = false;      // the batched router fits shared memory
     int mma_min_tok = 0;               // bucket size from which they run (0: never)
     __nv_bfloat16* h_pl = nullptr;     // [2][maxT * (k + 1)][maxI] h as bf16 hi / lo planes
     float* h_sum = nullptr;            // [maxT * (k + 1)][hsum_stride] group sums of h
@@ -423,6 +424,15 @@ extern "C" int moe_ctx_create(const MoeConfig* cfg, int max_tokens, moe_ctx** ou
     const int smem_router = (int)(H * sizeof(long long));
     if (e == cudaSuccess)
         e = raise_smem(k_router, smem_router);
+    if (e == cudaSuccess) {
+        int optin = 0;
+        e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, c->device);
+        const size_t rb = router_batch_smem(2, (int)H, (int)E);
+        if (e == cudaSuccess && rb <= (size_t)optin) {
+            e = raise_smem(k_router_batch<2>, (int)rb);
+            c->router_batch_ok = e == cudaSuccess;
+        }
+    }
     if (e == cudaSuccess)
         e = raise_smem(k_ffn_gateup_simple, (int)(H * sizeof(float)));
     if (e == cudaSuccess)
@@ -445,10 +455,19 @@ static int launch_router(moe_ctx* c, const int8_t* Wr, const moe_half* sc, const
                          const __half* x, int T, int32_t* idx, float* w, double* logits,
                          cudaStream_t s) {
     const MoeConfig& g = c->cfg;
+    double* lg = logits ? logits : c->logits;
+    if (T >= kRouterBatchMinTokens && c->router_batch_ok) {
+        // many tokens: digits once per token, the router matrix once per CTA
+        k_router_batch<2><<<(T + 1) / 2, kRouterBatchThreads, router_batch_smem(2, g.hidden, g.n_experts), s>>>(
+            Wr, reinterpret_cast<const __half*>(sc), bias, x, T, g.n_experts, g.hidden, g.top_k,
+            g.renorm, lg, idx, w);
+        CKL();
+        return MOE_OK;
+    }
     dim3 grid((g.n_experts + kRouterWarps - 1) / kRouterWarps, T);
     k_router<<<grid, 256, g.hidden * sizeof(long long), s>>>(
         Wr, reinterpret_cast<const __half*>(sc), bias, x, g.n_experts, g.hidden, g.top_k,
-        g.renorm, logits ? logits : c->logits, c->router_done, idx, w);
+        g.renorm, lg, c->router_done, idx, w);
     CKL();
     return MOE_OK;
 }
@@ -672,9 +691,13 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
             ta.y_pairs = c->y_pairs; ta.status = c->status;
         }
         const int chunks = (T + kGrpChunk - 1) / kGrpChunk;
-        k_gateup_grouped<false><<<dim3(I / 16, E), kGrpThreads, grouped_smem_gu(H), s>>>(
-            ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
-        CKL();
+        // with a threshold of one pair every routed bucket is on the tensor cores
+        const bool grp_routed = !(tc && tau <= 1);
+        if (grp_routed) {
+            k_gateup_grouped<false><<<dim3(I / 16, E), kGrpThreads, grouped_smem_gu(H), s>>>(
+                ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
+            CKL();
+        }
         if (!tc_shared) {
             k_gateup_grouped<true><<<dim3(Is / 16, 1, chunks), kGrpThreads, grouped_smem_gu(H), s>>>(
                 ex, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
@@ -689,9 +712,11 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
                 m_cgr, m_cgs, m_x[0], m_x[1], m_x[2], ex, stride, sh, gu);
             CKL();
         }
-        k_down_grouped<false><<<dim3(H / 16, E), kGrpThreads, grouped_smem_dn(I), s>>>(
-            ex, stride, sh, H, I, T, c->e_off, c->plist, cap, c->h_ws, c->maxI, c->y_pairs);
-        CKL();
+        if (grp_routed) {
+            k_down_grouped<false><<<dim3(H / 16, E), kGrpThreads, grouped_smem_dn(I), s>>>(
+                ex, stride, sh, H, I, T, c->e_off, c->plist, cap, c->h_ws, c->maxI, c->y_pairs);
+            CKL();
+        }
         if (!tc_shared) {
             k_down_grouped<true><<<dim3(H / 16, 1, chunks), kGrpThreads, grouped_smem_dn(Is), s>>>(
                 ex, stride, sh, H, Is, T, c->e_off, c->plist, cap, c->h_ws, c->maxI, c->y_pairs);

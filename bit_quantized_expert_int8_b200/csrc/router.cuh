@@ -20,100 +20,51 @@ namespace moeq4 {
 constexpr int kRouterWarps = 8;          // expert rows per CTA
 constexpr int kRouterDigits = 6;         // base-256 digits of |X| < 2^40 (6 * 8 > 40 + sign)
 
-// grid (ceil(E / 8), T), block 256, dynamic shared memory of at least
-// kRouterDigits * H bytes.  Each warp forms one logit; the last CTA
-// to finish a token selects its top-k and computes the routing weights.
-__global__ void __launch_bounds__(256)
-k_router(const int8_t* __restrict__ W, const __half* __restrict__ scale,
-         const float* __restrict__ bias, const __half* __restrict__ x,
-         int E, int H, int k, int renorm, double* __restrict__ logits,
-         int* __restrict__ done_counter, int32_t* __restrict__ topk_idx,
-         float* __restrict__ topk_w) {
-    extern __shared__ __align__(16) uint8_t sDig[];   // [kRouterDigits][H] digits of x * 2^24
-    __shared__ unsigned s_mx;
-    const int t = blockIdx.y;
-    const __half* xr = x + (size_t)t * H;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // digits needed for the largest |x| of this token
-    if (threadIdx.x == 0) s_mx = 0u;
-    __syncthreads();
-    float mx = 0.f;
-    for (int c = threadIdx.x; c < H; c += blockDim.x) mx = fmaxf(mx, fabsf(__half2float(xr[c])));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if (lane == 0) atomicMax(&s_mx, __float_as_uint(mx));   // non-negative floats order as integers
-    __syncthreads();
+// Digits needed for a token whose largest |x| is xmax_f (X = x * 2^24).
+__device__ __forceinline__ int router_ndigits(float xmax_f) {
     int NL = 1;
-    {
-        const double xmax = (double)__uint_as_float(s_mx) * 16777216.0;
-        double cap = 127.0;                           // largest |X| of NL digits: 127 (256^NL - 1) / 255
-        while (NL < kRouterDigits && xmax > cap) { NL++; cap = cap * 256.0 + 127.0; }
-    }
-    for (int c4 = threadIdx.x; c4 < H / 4; c4 += blockDim.x) {
-        uint32_t packed[kRouterDigits];
-#pragma unroll
-        for (int d = 0; d < kRouterDigits; d++) packed[d] = 0u;
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-            long long X = __float2ll_rn(__half2float(xr[4 * c4 + q]) * 16777216.0f);   // exact
-#pragma unroll
-            for (int d = 0; d < kRouterDigits; d++) {
-                const int digit = (int)((X + 128) & 255) - 128;
-                packed[d] |= (uint32_t)(digit & 255) << (8 * q);
-                X = (X - digit) >> 8;
-            }
-        }
-#pragma unroll
-        for (int d = 0; d < kRouterDigits; d++)
-            if (d < NL) reinterpret_cast<uint32_t*>(sDig + (size_t)d * H)[c4] = packed[d];
-    }
-    __syncthreads();
+    const double xmax = (double)xmax_f * 16777216.0;
+    double cap = 127.0;                               // largest |X| of NL digits: 127 (256^NL - 1) / 255
+    while (NL < kRouterDigits && xmax > cap) { NL++; cap = cap * 256.0 + 127.0; }
+    return NL;
+}
 
-    const int e = blockIdx.x * kRouterWarps + warp;
-    if (e < E) {
-        const int8_t* wr = W + (size_t)e * H;
-        int acc[kRouterDigits];
+// Four consecutive values of x (columns 4 c4 ..) as NL packed digit words:
+// digit d of X = x * 2^24 (balanced base 256) of value q in byte q of word d.
+__device__ __forceinline__ void router_digits4(const __half* xr, int c4, int NL, uint8_t* dig, int H) {
+    uint32_t packed[kRouterDigits];
 #pragma unroll
-        for (int d = 0; d < kRouterDigits; d++) acc[d] = 0;
-        for (int c0 = lane * 16; c0 < H; c0 += 32 * 16) {
-            const int4 v = *reinterpret_cast<const int4*>(wr + c0);
+    for (int d = 0; d < kRouterDigits; d++) packed[d] = 0u;
 #pragma unroll
-            for (int d = 0; d < kRouterDigits; d++) {
-                if (d < NL) {
-                    const int4 l = *reinterpret_cast<const int4*>(sDig + (size_t)d * H + c0);
-                    acc[d] = __dp4a(v.x, l.x, acc[d]);
-                    acc[d] = __dp4a(v.y, l.y, acc[d]);
-                    acc[d] = __dp4a(v.z, l.z, acc[d]);
-                    acc[d] = __dp4a(v.w, l.w, acc[d]);
-                }
-            }
-        }
-        long long S = 0;
+    for (int q = 0; q < 4; q++) {
+        long long X = __float2ll_rn(__half2float(xr[4 * c4 + q]) * 16777216.0f);   // exact
 #pragma unroll
-        for (int d = 0; d < kRouterDigits; d++)
-            if (d < NL) S += (long long)warp_sum(acc[d]) * (1ll << (8 * d));
-        if (lane == 0) {
-            double l = __ll2double_rn(S);
-            l = __dmul_rn(l, 0x1p-24);
-            l = __dmul_rn(l, (double)__half2float(scale[e]));
-            if (bias) l = __dadd_rn(l, (double)bias[e]);
-            logits[(size_t)t * E + e] = l;
+        for (int d = 0; d < kRouterDigits; d++) {
+            const int digit = (int)((X + 128) & 255) - 128;
+            packed[d] |= (uint32_t)(digit & 255) << (8 * q);
+            X = (X - digit) >> 8;
         }
     }
+#pragma unroll
+    for (int d = 0; d < kRouterDigits; d++)
+        if (d < NL) reinterpret_cast<uint32_t*>(dig + (size_t)d * H)[c4] = packed[d];
+}
 
-    // Last CTA of this token does the selection.
-    __shared__ int s_last;
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int prev = atomicAdd(&done_counter[t], 1);
-        s_last = (prev == (int)gridDim.x - 1);
-    }
-    __syncthreads();
-    if (!s_last || warp != 0) return;
-    __threadfence();
+// Logit of expert e from its exact integer row sum S = sum_c W[e][c] X[c].
+__device__ __forceinline__ double router_logit(long long S, const __half* scale, const float* bias, int e) {
+    double l = __ll2double_rn(S);
+    l = __dmul_rn(l, 0x1p-24);
+    l = __dmul_rn(l, (double)__half2float(scale[e]));
+    if (bias) l = __dadd_rn(l, (double)bias[e]);
+    return l;
+}
 
-    const volatile double* lg = logits + (size_t)t * E;
+// Top-k of one token's E logits by one warp (largest value, lowest index on
+// ties), then the softmax over all E logits in fp64 and the selected
+// probabilities (renormalised over the k when renorm).
+template <typename LP>
+__device__ __forceinline__ void router_select(LP lg, int E, int k, int renorm, int lane,
+                                              int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
     constexpr int kPer = MOE_MAX_EXPERTS / 32;        // logits per lane
     double v[kPer];
     bool taken[kPer];
@@ -159,11 +110,201 @@ k_router(const int8_t* __restrict__ W, const __half* __restrict__ scale,
         double p[MOE_MAX_TOPK], zs = 0.0;
         for (int j = 0; j < k; j++) { p[j] = exp(sel_l[j] - m) / z; zs += p[j]; }
         for (int j = 0; j < k; j++) {
-            topk_idx[(size_t)t * k + j] = sel[j];
-            topk_w[(size_t)t * k + j] = (float)(renorm ? p[j] / zs : p[j]);
+            topk_idx[j] = sel[j];
+            topk_w[j] = (float)(renorm ? p[j] / zs : p[j]);
         }
+    }
+}
+
+// grid (ceil(E / 8), T), block 256, dynamic shared memory of at least
+// kRouterDigits * H bytes.  Each warp forms one logit; the last CTA
+// to finish a token selects its top-k and computes the routing weights.
+__global__ void __launch_bounds__(256)
+k_router(const int8_t* __restrict__ W, const __half* __restrict__ scale,
+         const float* __restrict__ bias, const __half* __restrict__ x,
+         int E, int H, int k, int renorm, double* __restrict__ logits,
+         int* __restrict__ done_counter, int32_t* __restrict__ topk_idx,
+         float* __restrict__ topk_w) {
+    extern __shared__ __align__(16) uint8_t sDig[];   // [kRouterDigits][H] digits of x * 2^24
+    __shared__ unsigned s_mx;
+    const int t = blockIdx.y;
+    const __half* xr = x + (size_t)t * H;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // digits needed for the largest |x| of this token
+    if (threadIdx.x == 0) s_mx = 0u;
+    __syncthreads();
+    float mx = 0.f;
+    for (int c = threadIdx.x; c < H; c += blockDim.x) mx = fmaxf(mx, fabsf(__half2float(xr[c])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) atomicMax(&s_mx, __float_as_uint(mx));   // non-negative floats order as integers
+    __syncthreads();
+    const int NL = router_ndigits(__uint_as_float(s_mx));
+    for (int c4 = threadIdx.x; c4 < H / 4; c4 += blockDim.x) router_digits4(xr, c4, NL, sDig, H);
+    __syncthreads();
+
+    const int e = blockIdx.x * kRouterWarps + warp;
+    if (e < E) {
+        const int8_t* wr = W + (size_t)e * H;
+        int acc[kRouterDigits];
+#pragma unroll
+        for (int d = 0; d < kRouterDigits; d++) acc[d] = 0;
+        for (int c0 = lane * 16; c0 < H; c0 += 32 * 16) {
+            const int4 v = *reinterpret_cast<const int4*>(wr + c0);
+#pragma unroll
+            for (int d = 0; d < kRouterDigits; d++) {
+                if (d < NL) {
+                    const int4 l = *reinterpret_cast<const int4*>(sDig + (size_t)d * H + c0);
+                    acc[d] = __dp4a(v.x, l.x, acc[d]);
+                    acc[d] = __dp4a(v.y, l.y, acc[d]);
+                    acc[d] = __dp4a(v.z, l.z, acc[d]);
+                    acc[d] = __dp4a(v.w, l.w, acc[d]);
+                }
+            }
+        }
+        long long S = 0;
+#pragma unroll
+        for (int d = 0; d < kRouterDigits; d++)
+            if (d < NL) S += (long long)warp_sum(acc[d]) * (1ll << (8 * d));
+        if (lane == 0) logits[(size_t)t * E + e] = router_logit(S, scale, bias, e);
+    }
+
+    // Last CTA of this token does the selection.
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int prev = atomicAdd(&done_counter[t], 1);
+        s_last = (prev == (int)gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!s_last || warp != 0) return;
+    __threadfence();
+
+    const volatile double* lg = logits + (size_t)t * E;
+    router_select(lg, E, k, renorm, lane, topk_idx + (size_t)t * k, topk_w + (size_t)t * k);
+    if (lane == 0) {
         done_counter[t] = 0;                          // ready for the next launch
     }
+}
+
+// Steps of many tokens: one CTA per TB tokens and every expert, so a
+// token's digits are formed once and the router matrix is read once per CTA.
+// Each warp takes expert rows two at a time (lanes read consecutive 16-byte
+// chunks of the rows, several chunks in flight) and reduces its TB x NL digit
+// sums across the lanes.  The
+// arithmetic (digits, exact integer row sums, fp64 logits, selection) is that
+// of k_router, so the two kernels choose the same experts with the same
+// weights.  grid ceil(T / TB), block kRouterBatchThreads, dynamic shared
+// memory router_batch_smem(TB, H, E).
+constexpr int kRouterBatchThreads = 512;
+constexpr int kRouterBatchMinTokens = 128;  // steps from which the batched router runs (measured)
+__host__ __device__ constexpr size_t router_batch_smem(int TB, int H, int E) {
+    return (size_t)TB * kRouterDigits * H + (size_t)TB * E * sizeof(double);
+}
+template <int TB>
+__global__ void __launch_bounds__(kRouterBatchThreads)
+k_router_batch(const int8_t* __restrict__ W, const __half* __restrict__ scale,
+               const float* __restrict__ bias, const __half* __restrict__ x, int T, int E, int H,
+               int k, int renorm, double* __restrict__ logits, int32_t* __restrict__ topk_idx,
+               float* __restrict__ topk_w) {
+    extern __shared__ __align__(16) uint8_t sDig[];   // [TB][kRouterDigits][H], then [TB][E] fp64
+    double* sLg = reinterpret_cast<double*>(sDig + (size_t)TB * kRouterDigits * H);
+    __shared__ unsigned s_mx[TB];
+    const int t0 = blockIdx.x * TB, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nt = min(TB, T - t0);
+    if (tid < TB) s_mx[tid] = 0u;
+    __syncthreads();
+    for (int t = 0; t < nt; t++) {
+        const __half* xr = x + (size_t)(t0 + t) * H;
+        float mx = 0.f;
+        for (int c = tid; c < H; c += blockDim.x) mx = fmaxf(mx, fabsf(__half2float(xr[c])));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) atomicMax(&s_mx[t], __float_as_uint(mx));
+    }
+    __syncthreads();
+    int NL[TB];
+#pragma unroll
+    for (int t = 0; t < TB; t++) NL[t] = t < nt ? router_ndigits(__uint_as_float(s_mx[t])) : 0;
+    for (int t = 0; t < nt; t++) {
+        const __half* xr = x + (size_t)(t0 + t) * H;
+        for (int c4 = tid; c4 < H / 4; c4 += blockDim.x)
+            router_digits4(xr, c4, NL[t], sDig + (size_t)t * kRouterDigits * H, H);
+    }
+    __syncthreads();
+    // two expert rows per warp pass, up to 6 chunks of 16 bytes per lane and
+    // row in flight before their dot products
+    constexpr int kCh = 6;
+    for (int e0 = 2 * warp; e0 < E; e0 += 2 * (kRouterBatchThreads / 32)) {
+        const bool two = e0 + 1 < E;
+        const int8_t* wr0 = W + (size_t)e0 * H;
+        const int8_t* wr1 = W + (size_t)(two ? e0 + 1 : e0) * H;
+        int acc[2][TB][kRouterDigits];
+#pragma unroll
+        for (int r = 0; r < 2; r++)
+#pragma unroll
+            for (int t = 0; t < TB; t++)
+#pragma unroll
+                for (int d = 0; d < kRouterDigits; d++) acc[r][t][d] = 0;
+        for (int cb = lane * 16; cb < H; cb += kCh * 32 * 16) {
+            int4 w[2][kCh];
+#pragma unroll
+            for (int i = 0; i < kCh; i++) {
+                const int c0 = cb + i * 32 * 16;
+                if (c0 < H) {
+                    w[0][i] = *reinterpret_cast<const int4*>(wr0 + c0);
+                    w[1][i] = *reinterpret_cast<const int4*>(wr1 + c0);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kCh; i++) {
+                const int c0 = cb + i * 32 * 16;
+                if (c0 < H) {
+#pragma unroll
+                    for (int t = 0; t < TB; t++) {
+#pragma unroll
+                        for (int d = 0; d < kRouterDigits; d++) {
+                            if (d < NL[t]) {
+                                const int4 l = *reinterpret_cast<const int4*>(
+                                    sDig + ((size_t)t * kRouterDigits + d) * H + c0);
+#pragma unroll
+                                for (int r = 0; r < 2; r++) {
+                                    acc[r][t][d] = __dp4a(w[r][i].x, l.x, acc[r][t][d]);
+                                    acc[r][t][d] = __dp4a(w[r][i].y, l.y, acc[r][t][d]);
+                                    acc[r][t][d] = __dp4a(w[r][i].z, l.z, acc[r][t][d]);
+                                    acc[r][t][d] = __dp4a(w[r][i].w, l.w, acc[r][t][d]);
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 2; r++) {
+            if (r == 1 && !two) break;
+            const int e = e0 + r;
+#pragma unroll
+            for (int t = 0; t < TB; t++) {
+                if (t < nt) {
+                    long long S = 0;
+#pragma unroll
+                    for (int d = 0; d < kRouterDigits; d++)
+                        if (d < NL[t]) S += (long long)warp_sum(acc[r][t][d]) * (1ll << (8 * d));
+                    if (lane == 0) {
+                        const double l = router_logit(S, scale, bias, e);
+                        sLg[t * E + e] = l;
+                        logits[(size_t)(t0 + t) * E + e] = l;
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (warp < nt)
+        router_select(sLg + warp * E, E, k, renorm, lane, topk_idx + (size_t)(t0 + warp) * k,
+                      topk_w + (size_t)(t0 + warp) * k);
 }
 
 }  // namespace moeq4

@@ -124,7 +124,7 @@ int moe_set_wait_ns(moe_ctx *ctx, unsigned long long ns);
  * bf16 planes; fp32 accumulation, one accumulator per 64-column group folded
  * with its scale and bias); the other buckets, and every bucket of a smaller
  * step, run on the CUDA-core grouped kernels.  min_tokens = 0 keeps every
- * bucket on the CUDA cores.  The default is 4 where the shape allows the
+ * bucket on the CUDA cores.  The default is 1 where the shape allows the
  * tensor-core kernels (hidden a multiple of 128, the staging buffers within
  * shared memory), else 0.  Host call, no device work.  Returns
  * MOE_ERR_INVALID_ARG for min_tokens < 0 and MOE_ERR_UNSUPPORTED_SHAPE for

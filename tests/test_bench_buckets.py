@@ -17,8 +17,10 @@ def test_bucket_split_rules():
     counts = [0, 1, 3, 4, 5, 40, 0, 2]
     # small step: everything on the grouped kernels
     assert b.bucket_split(counts, T=8) == (0, 6)
-    # large step: buckets of >= 4 pairs on tcgen05
-    assert b.bucket_split(counts, T=32) == (3, 3)
+    # large step: by default every used bucket on tcgen05
+    assert b.bucket_split(counts, T=32) == (6, 0)
+    # a threshold of 4 pairs leaves the smaller buckets on the grouped kernels
+    assert b.bucket_split(counts, T=32, min_tokens=4) == (3, 3)
     assert b.bucket_split(counts, T=256, min_tokens=1) == (6, 0)
     assert b.bucket_split(counts, T=256, min_tokens=0) == (0, 6)
     assert b.bucket_split([0] * 16, T=64) == (0, 0)

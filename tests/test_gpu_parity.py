@@ -34,8 +34,11 @@ def ctx_for(cfg, T=1):
 
 # ---------------------------------------------------------------- router ----
 
+# T >= 128 runs the batched router (one CTA per two tokens, every expert);
+# 131 tokens leave a CTA with one token.
 @pytest.mark.parametrize("cfg,T,bias", [(TINY, 1, None), (TINY, 7, 1.5), (SMALL, 3, 0.7),
-                                        (LAYER, 4, None), (LAYER, 2, 1.5)])
+                                        (LAYER, 4, None), (LAYER, 2, 1.5), (TINY, 33, 1.5),
+                                        (LAYER, 64, None), (LAYER, 131, 1.5), (TINY, 128, None)])
 def test_router_parity(cfg, T, bias):
     L = make_layer(cfg, seed=3, bias_std=bias)
     x = synth.tokens(T, cfg.H, seed=5, device=DEV)
