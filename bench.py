@@ -296,6 +296,8 @@ TRAFFIC_BY_SOURCE = {
     "ab523b1bf6c48f302f20a8d0fa33bdea867f6816a4e0a6fbc4a69b12422ad079": 37327872,
     # the same capture with 24-bit x digits: read 37,290,496 + write 114,432
     "c31f5378bd41ff1c3afc7da62ad3dfbbf79f3cba4022471fda56907f7fdcafba": 37404928,
+    # status word read only by waits longer than 20 us: read 37,290,240 + write 140,544
+    "315e1cae13a9292cedfd34824b3dfbd1020a3c725007f273bb51283915d59fcb": 37430784,
 }
 
 
