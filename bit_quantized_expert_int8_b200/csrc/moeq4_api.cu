@@ -15,6 +15,7 @@
 
 #include "common.cuh"
 #include "ffn_tc.cuh"
+#include "ep.cuh"
 #include "ffn_simple.cuh"
 #include "grouped.cuh"
 #include "layer_fused.cuh"
@@ -599,6 +600,75 @@ extern "C" int moe_combine(moe_ctx* c, const float* y_routed, const float* y_sha
                           reinterpret_cast<__half*>(residual), stream);
 }
 
+static int ffn_grouped(moe_ctx* c, const uint8_t* ex, int E, const uint8_t* sh, const __half* xin,
+                       const int32_t* idx, int T, int k, cudaStream_t s);
+
+extern "C" int moe_ep_dispatch(moe_ctx* c, const int32_t* topk_idx, int T, int n_ranks,
+                               const moe_half* x, moe_half* send_x, int32_t* send_expert,
+                               int32_t* send_order, int32_t* send_counts, moe_stream_t stream) {
+    if (!c || !topk_idx || !x || !send_x || !send_expert || !send_order || !send_counts)
+        return fail(MOE_ERR_INVALID_ARG, "moe_ep_dispatch: NULL argument");
+    const MoeConfig& g = c->cfg;
+    if (T < 1 || T > c->maxT) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T=%d outside 1..%d", T, c->maxT);
+    if (n_ranks < 1 || n_ranks > 32 || g.n_experts % n_ranks)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n_ranks=%d must divide n_experts=%d (at most 32)",
+                    n_ranks, g.n_experts);
+    if (!aligned4(topk_idx) || !aligned16(x) || !aligned16(send_x) || !aligned4(send_expert) ||
+        !aligned4(send_order) || !aligned4(send_counts))
+        return fail(MOE_ERR_ALIGNMENT, "moe_ep_dispatch: misaligned pointer");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int P = T * g.top_k, epr = g.n_experts / n_ranks;
+    k_ep_plan<<<1, 32 * n_ranks, 0, s>>>(topk_idx, P, g.n_experts, epr, n_ranks, send_counts, send_order,
+                                          c->status);
+    CKL();
+    k_ep_gather<<<(P + 7) / 8, 256, 0, s>>>(reinterpret_cast<const __half*>(x), topk_idx, send_order, P,
+                                             g.top_k, g.hidden, epr, reinterpret_cast<__half*>(send_x),
+                                             send_expert);
+    CKL();
+    return MOE_OK;
+}
+
+extern "C" int moe_ffn_rows(moe_ctx* c, const void* experts, int n_experts, const int32_t* expert_of_row,
+                            int R, const moe_half* x_rows, float* y_rows, moe_stream_t stream) {
+    if (!c || !experts || !expert_of_row || !x_rows || !y_rows)
+        return fail(MOE_ERR_INVALID_ARG, "moe_ffn_rows: NULL argument");
+    const MoeConfig& g = c->cfg;
+    if (n_experts < 1 || n_experts > g.n_experts)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n_experts=%d outside 1..%d", n_experts, g.n_experts);
+    // the rows take the place of R tokens with one pair each: 2 R workspace rows
+    const int rmax = std::min(c->maxT * g.top_k, c->maxT * (g.top_k + 1) / 2);
+    if (R < 0 || R > rmax)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "R=%d outside 0..%d (the context's max_tokens holds "
+                    "min(max_tokens * top_k, max_tokens * (top_k + 1) / 2) rows)", R, rmax);
+    if (!c->grouped_ok)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_ffn_rows needs the grouped kernels for this shape");
+    if (!aligned16(experts) || !aligned4(expert_of_row) || !aligned16(x_rows) || !aligned16(y_rows))
+        return fail(MOE_ERR_ALIGNMENT, "moe_ffn_rows: misaligned pointer");
+    if (R == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // each row is its own token choosing one expert: rows T + q of the pair outputs
+    TRY(ffn_grouped(c, static_cast<const uint8_t*>(experts), n_experts, nullptr,
+                    reinterpret_cast<const __half*>(x_rows), expert_of_row, R, 1, s));
+    CK(cudaMemcpyAsync(y_rows, c->y_pairs + (size_t)R * g.hidden, (size_t)R * g.hidden * sizeof(float),
+                       cudaMemcpyDeviceToDevice, s));
+    return MOE_OK;
+}
+
+extern "C" int moe_ep_unpermute(moe_ctx* c, const float* y_sorted, const int32_t* send_order, int n,
+                                float* y_pairs, moe_stream_t stream) {
+    if (!c || !y_sorted || !send_order || !y_pairs)
+        return fail(MOE_ERR_INVALID_ARG, "moe_ep_unpermute: NULL argument");
+    if (n < 0 || n > c->maxT * c->cfg.top_k)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n=%d outside 0..%d", n, c->maxT * c->cfg.top_k);
+    if (!aligned16(y_sorted) || !aligned4(send_order) || !aligned16(y_pairs))
+        return fail(MOE_ERR_ALIGNMENT, "moe_ep_unpermute: misaligned pointer");
+    if (n == 0) return MOE_OK;
+    k_ep_unpermute<<<(n + 7) / 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(y_sorted, send_order, n,
+                                                                                 c->cfg.hidden, y_pairs);
+    CKL();
+    return MOE_OK;
+}
+
 extern "C" int moe_lfu_init(moe_ctx* c, MoeLfuTable* table, int n_slots, moe_stream_t stream) {
     if (!c || !table) return fail(MOE_ERR_INVALID_ARG, "moe_lfu_init: NULL argument");
     if (n_slots <= c->cfg.top_k || n_slots > MOE_MAX_SLOTS)
@@ -623,45 +693,25 @@ extern "C" int moe_cache_lookup_lfu(moe_ctx* c, MoeLfuTable* table, const int32_
     return MOE_OK;
 }
 
-// Resident layer body on one stream (also used inside the stack capture).
-static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const MoeLayerOut* o,
-                          int flags, cudaStream_t s) {
-    const MoeConfig& g = c->cfg;
-    const int k = g.top_k, H = g.hidden;
-    if (T == 1 && c->fused_ok) {
-        const bool pre = (flags & MOE_PRENORM) != 0;
-        TRY(launch_fused(c, L, x, pre ? c->h_alt : nullptr,
-                         reinterpret_cast<__half*>(o->x_norm), o->y, o->topk_idx, o->topk_w,
-                         pre ? 1 : 0, s));
-        if (pre) {
-            k_copy_rows<<<1, 256, 0, s>>>(c->h_alt, x, H);
-            CKL();
-        }
-        return MOE_OK;
-    }
-    const __half* xin = x;
-    __half* xn = o->x_norm ? reinterpret_cast<__half*>(o->x_norm) : c->x_norm;
-    if (flags & MOE_PRENORM) {
-        k_rmsnorm<<<T, 256, 0, s>>>(x, xn, H, g.rms_eps);
-        CKL();
-        xin = xn;
-    }
-    int32_t* idx = o->topk_idx ? o->topk_idx : c->idx;
-    float* w = o->topk_w ? o->topk_w : c->w;
-    TRY(launch_router(c, L->router_w, L->router_scale, L->router_bias, xin, T, idx, w, nullptr, s));
-    const size_t stride = BlobLayout(H, g.inter).bytes;
-    const int P = T * (k + 1);
-    if (c->grouped_ok) {
-        // each expert read once for all of its tokens
-        const uint8_t* ex = static_cast<const uint8_t*>(L->experts);
-        const uint8_t* sh = static_cast<const uint8_t*>(L->shared_blob);
-        const int E = g.n_experts, I = g.inter, Is = g.inter_shared;
+// Multi-token FFNs of all experts resident (T >= 1 tokens, k pairs each,
+// pair q = t * k + j choosing idx[q] < E): outputs in c->y_pairs, row t for
+// the shared expert (when sh is given) and row T + q for pair q.  Each expert
+// is read once for all of its tokens.
+static int ffn_grouped(moe_ctx* c, const uint8_t* ex, int E, const uint8_t* sh, const __half* xin,
+                       const int32_t* idx, int T, int k, cudaStream_t s) {
+    {
+        const MoeConfig& g = c->cfg;
+        const int H = g.hidden;
+        const size_t stride = BlobLayout(H, g.inter).bytes;
+        const int I = g.inter, Is = g.inter_shared;
+        const bool with_shared = sh != nullptr;
+        if (!with_shared) sh = ex;                    // shared-expert maps: encoded, never read
         // In steps of at least kMmaMinStep tokens, routed buckets of tau or more
         // pairs and the shared expert (T >= tau) run on the tensor cores
         // (tau = 0: none); the rest on the CUDA-core grouped kernels.
         const int tau = c->mma_ok ? c->mma_min_tok : 0;
         const bool tc = tau > 0 && T >= kMmaMinStep;
-        const bool tc_shared = tc && T >= tau;
+        const bool tc_shared = with_shared && tc && T >= tau;
         const int cap = tc ? tau : 0x7fffffff;
         const int P = T * (k + 1), hs = c->maxI;
         __nv_bfloat16 *hh = c->h_pl, *hl = c->h_pl + (size_t)P * hs;
@@ -698,7 +748,7 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
                 ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
             CKL();
         }
-        if (!tc_shared) {
+        if (with_shared && !tc_shared) {
             k_gateup_grouped<true><<<dim3(Is / 16, 1, chunks), kGrpThreads, grouped_smem_gu(H), s>>>(
                 ex, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
             CKL();
@@ -717,7 +767,7 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
                 ex, stride, sh, H, I, T, c->e_off, c->plist, cap, c->h_ws, c->maxI, c->y_pairs);
             CKL();
         }
-        if (!tc_shared) {
+        if (with_shared && !tc_shared) {
             k_down_grouped<true><<<dim3(H / 16, 1, chunks), kGrpThreads, grouped_smem_dn(Is), s>>>(
                 ex, stride, sh, H, Is, T, c->e_off, c->plist, cap, c->h_ws, c->maxI, c->y_pairs);
             CKL();
@@ -731,6 +781,42 @@ static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const
                 m_cdr, m_cds, m_h[0], m_h[1], m_h[2], ex, stride, sh, dn);
             CKL();
         }
+    }
+    return MOE_OK;
+}
+
+// Resident layer body on one stream (also used inside the stack capture).
+static int layer_resident(moe_ctx* c, const MoeLayer* L, __half* x, int T, const MoeLayerOut* o,
+                          int flags, cudaStream_t s) {
+    const MoeConfig& g = c->cfg;
+    const int k = g.top_k, H = g.hidden;
+    if (T == 1 && c->fused_ok) {
+        const bool pre = (flags & MOE_PRENORM) != 0;
+        TRY(launch_fused(c, L, x, pre ? c->h_alt : nullptr,
+                         reinterpret_cast<__half*>(o->x_norm), o->y, o->topk_idx, o->topk_w,
+                         pre ? 1 : 0, s));
+        if (pre) {
+            k_copy_rows<<<1, 256, 0, s>>>(c->h_alt, x, H);
+            CKL();
+        }
+        return MOE_OK;
+    }
+    const __half* xin = x;
+    __half* xn = o->x_norm ? reinterpret_cast<__half*>(o->x_norm) : c->x_norm;
+    if (flags & MOE_PRENORM) {
+        k_rmsnorm<<<T, 256, 0, s>>>(x, xn, H, g.rms_eps);
+        CKL();
+        xin = xn;
+    }
+    int32_t* idx = o->topk_idx ? o->topk_idx : c->idx;
+    float* w = o->topk_w ? o->topk_w : c->w;
+    TRY(launch_router(c, L->router_w, L->router_scale, L->router_bias, xin, T, idx, w, nullptr, s));
+    const size_t stride = BlobLayout(H, g.inter).bytes;
+    const int P = T * (k + 1);
+    if (c->grouped_ok) {
+        // each expert read once for all of its tokens
+        TRY(ffn_grouped(c, static_cast<const uint8_t*>(L->experts), g.n_experts,
+                        static_cast<const uint8_t*>(L->shared_blob), xin, idx, T, k, s));
     } else {
         k_build_pairs<<<(P + 127) / 128, 128, 0, s>>>(L->shared_blob, g.inter_shared,
                                                       static_cast<const uint8_t*>(L->experts), stride,

@@ -31,6 +31,7 @@ MOE_MAX_SLOTS = 32
 EXPORTS = ("moe_ctx_create", "moe_ctx_destroy", "moe_ctx_check", "moe_ctx_trace", "moe_ctx_info",
            "moe_last_error", "moe_blob_bytes",
            "moe_router_topk", "moe_expert_ffn_q4", "moe_combine", "moe_lfu_init",
+           "moe_ep_dispatch", "moe_ffn_rows", "moe_ep_unpermute",
            "moe_cache_lookup_lfu", "moe_layer_decode", "moe_stack_decode",
            "moe_router_topk_noalloc", "moe_set_mma_min_tokens", "moe_set_wait_ns",
            "moe_store_stride", "moe_store_open", "moe_store_close", "moe_store_read",
@@ -101,6 +102,9 @@ def load() -> ctypes.CDLL:
         "moe_router_topk": ([P, P, P, P, P, i32, P, P, P, P], i32),
         "moe_expert_ffn_q4": ([P, P, i32, P, i32, P, P], i32),
         "moe_combine": ([P, P, P, P, i32, P, P, P], i32),
+        "moe_ep_dispatch": ([P, P, i32, i32, P, P, P, P, P, P], i32),
+        "moe_ffn_rows": ([P, P, i32, P, i32, P, P, P], i32),
+        "moe_ep_unpermute": ([P, P, P, i32, P, P], i32),
         "moe_lfu_init": ([P, P, i32, P], i32),
         "moe_cache_lookup_lfu": ([P, P, P, i32, P, P, P, P], i32),
         "moe_layer_decode": ([P, ctypes.POINTER(CMoeLayer), P, i32,
@@ -246,6 +250,23 @@ def moe_expert_ffn_q4(ctx, pairs, n_pairs, x, T, y, stream=None):
 def moe_combine(ctx, y_routed, y_shared, topk_w, T, y_out, residual=None, stream=None):
     _check(load().moe_combine(ctx.handle, _ptr(y_routed), _ptr(y_shared), _ptr(topk_w), T,
                               _ptr(y_out), _ptr(residual), _stream(stream)))
+
+
+def moe_ep_dispatch(ctx, topk_idx, T, n_ranks, x, send_x, send_expert, send_order, send_counts,
+                    stream=None):
+    _check(load().moe_ep_dispatch(ctx.handle, _ptr(topk_idx), T, n_ranks, _ptr(x), _ptr(send_x),
+                                  _ptr(send_expert), _ptr(send_order), _ptr(send_counts),
+                                  _stream(stream)))
+
+
+def moe_ffn_rows(ctx, experts, n_experts, expert_of_row, R, x_rows, y_rows, stream=None):
+    _check(load().moe_ffn_rows(ctx.handle, _ptr(experts), n_experts, _ptr(expert_of_row), R,
+                               _ptr(x_rows), _ptr(y_rows), _stream(stream)))
+
+
+def moe_ep_unpermute(ctx, y_sorted, send_order, n, y_pairs, stream=None):
+    _check(load().moe_ep_unpermute(ctx.handle, _ptr(y_sorted), _ptr(send_order), n, _ptr(y_pairs),
+                                   _stream(stream)))
 
 
 def new_lfu_table(device="cuda"):

@@ -248,6 +248,44 @@ typedef struct {
 int moe_expert_ffn_q4(moe_ctx *ctx, const MoeFfnPair *pairs, int n_pairs,
                       const moe_half *x, int T, float *y, moe_stream_t stream);
 
+/* ------------------------------------------------- expert parallel ----
+ * Experts partitioned over n_ranks ranks (rank r owns experts
+ * r * E / n_ranks .. (r + 1) * E / n_ranks - 1); each rank routes its own
+ * tokens and sends every (token, expert) pair to the expert's owner, which
+ * applies the expert and sends the row back.  The pages run one process on
+ * one machine; this is the B200 scale-out reading of their per-expert FFN
+ * step ([LH] 04 pipeline steps 2-3, one expert applied to the rows routed to
+ * it).  The host exchanges the rows between the calls (two all-to-alls).
+ *
+ * moe_ep_dispatch: the T * top_k pairs of topk_idx (device int32 [T][k])
+ * sorted by destination rank, pairs in index order within a destination:
+ *   send_counts  device int32 [n_ranks]: pairs for each rank;
+ *   send_order   device int32 [T * k]: pair index q = t * k + j per position;
+ *   send_x       device fp16 [T * k][H]: x[q / k] per position (x [T][H]);
+ *   send_expert  device int32 [T * k]: the expert's index at its owner.
+ * n_ranks must divide n_experts (at most 32).  An expert index outside
+ * [0, n_experts) is not sent and moe_ctx_check reports MOE_ERR_INVALID_ARG. */
+int moe_ep_dispatch(moe_ctx *ctx, const int32_t *topk_idx, int T, int n_ranks,
+                    const moe_half *x, moe_half *send_x, int32_t *send_expert,
+                    int32_t *send_order, int32_t *send_counts, moe_stream_t stream);
+
+/* moe_ffn_rows: R rows, row r through expert expert_of_row[r] of the
+ * n_experts blobs at `experts` (device, blob stride moe_blob_bytes(H, I)):
+ * y_rows[r] = down(GELU(gate x_r) * up x_r), the grouped / tensor-core
+ * kernels of the multi-token path with each row its own token.
+ *   expert_of_row device int32 [R]; x_rows device fp16 [R][H];
+ *   y_rows device fp32 [R][H].
+ * R must be 0..min(max_tokens * top_k, max_tokens * (top_k + 1) / 2) (each
+ * row takes a token's and a pair's place in the context's workspace; R = 0
+ * does nothing); larger R returns MOE_ERR_UNSUPPORTED_SHAPE. */
+int moe_ffn_rows(moe_ctx *ctx, const void *experts, int n_experts, const int32_t *expert_of_row,
+                 int R, const moe_half *x_rows, float *y_rows, moe_stream_t stream);
+
+/* moe_ep_unpermute: rows returned in send order back to pair order,
+ * y_pairs[send_order[p]] = y_sorted[p] for p < n (device fp32 rows of H). */
+int moe_ep_unpermute(moe_ctx *ctx, const float *y_sorted, const int32_t *send_order, int n,
+                     float *y_pairs, moe_stream_t stream);
+
 /* --------------------------------------------------------- combine ----
  * [LH] "Concurrence pour masquer la latence", [RM] "L'affirmation des 2 Go
  * ...": the shared and routed outputs combine,
