@@ -691,6 +691,20 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
     griddep_wait();
     constexpr int kHPer = 16;                    // h values per thread (H <= 4096)
     if (a.prenorm) {
+        // residual row of this CTA's routed down items (for the final h + y),
+        // loaded with the input so that both round trips overlap
+        __half hres = __float2half(0.f);
+        int hres_t = -1;
+        if (a.NRD > 0 && tid < kMaxDownItems * kRdRows) {
+            const int d0 = a.NR + a.NSG + a.NSD + a.NRG;
+            int q0 = blockIdx.x;
+            while (q0 < d0) q0 += gridDim.x;
+            const int q = q0 + (tid / kRdRows) * gridDim.x;
+            if (q < a.NTOT) {
+                hres_t = tid;
+                hres = __ushort_as_half(__ldcg((const unsigned short*)a.x_in + kRdRows * (q - d0) + (tid % kRdRows)));
+            }
+        }
         __half hv[kHPer];
         unsigned __int128 acc = 0;
 #pragma unroll
@@ -704,35 +718,22 @@ __device__ __forceinline__ void fused_consumers(const FusedArgs& a, uint8_t* sta
         acc = warp_sum_u128(acc);
         if (lane == 0) { sc[2 * warp] = (unsigned long long)(acc >> 64); sc[2 * warp + 1] = (unsigned long long)acc; }
         named_bar(1, nthr);
-        if (tid == 0) {
+        // every thread forms the same exact total and the same 1 / rms
+        double r;
+        {
             unsigned __int128 tot = 0;
             for (int w = 0; w < kFusedConsumerWarps; w++)
                 tot += ((unsigned __int128)sc[2 * w] << 64) | sc[2 * w + 1];
             const double s = __dmul_rn(u128_to_double_rn(tot), 0x1p-48);
             const double ms = __ddiv_rn(s, (double)H);
-            const double r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms, a.eps)));
-            sc[16] = (unsigned long long)__double_as_longlong(r);
+            r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms, a.eps)));
         }
-        named_bar(1, nthr);
-        const double r = __longlong_as_double((long long)sc[16]);
 #pragma unroll
         for (int i = 0; i < kHPer; i++) {
             const int c = tid + nthr * i;
             if (c < H) xs[c] = __double2half(__dmul_rn((double)__half2float(hv[i]), r));
         }
-        // residual rows of this CTA's routed down items, for the final h + y
-        if (a.NRD > 0) {
-            const int d0 = a.NR + a.NSG + a.NSD + a.NRG;
-            int q0 = blockIdx.x;
-            while (q0 < d0) q0 += gridDim.x;
-            for (int t = tid; t < kMaxDownItems * kRdRows; t += nthr) {
-                const int q = q0 + (t / kRdRows) * gridDim.x;
-                if (q < a.NTOT) {
-                    const int row = kRdRows * (q - d0) + (t % kRdRows);
-                    cs->h_rows[t] = __ushort_as_half(__ldcg((const unsigned short*)a.x_in + row));
-                }
-            }
-        }
+        if (hres_t >= 0) cs->h_rows[hres_t] = hres;
     } else {
         for (int c = tid; c < H / 8; c += nthr)
             reinterpret_cast<uint4*>(xs)[c] = __ldcg(reinterpret_cast<const uint4*>(a.x_in) + c);
