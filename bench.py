@@ -298,6 +298,8 @@ TRAFFIC_BY_SOURCE = {
     "c31f5378bd41ff1c3afc7da62ad3dfbbf79f3cba4022471fda56907f7fdcafba": 37404928,
     # status word read only by waits longer than 20 us: read 37,290,240 + write 140,544
     "315e1cae13a9292cedfd34824b3dfbd1020a3c725007f273bb51283915d59fcb": 37430784,
+    # pre-norm with the down items' residual rows loaded beside x: read 37,289,984 + write 34,048
+    "48bcc63c17dd9b2c08b20c7ddc1217797a982fe5d4bfbf3c4657e479a352f572": 37324032,
 }
 
 
