@@ -459,9 +459,16 @@ static int launch_router(moe_ctx* c, const int8_t* Wr, const moe_half* sc, const
     double* lg = logits ? logits : c->logits;
     if (T >= kRouterBatchMinTokens && c->router_batch_ok) {
         // many tokens: digits once per token, the router matrix once per CTA
-        k_router_batch<2><<<(T + 1) / 2, kRouterBatchThreads, router_batch_smem(2, g.hidden, g.n_experts), s>>>(
+        // expert blocks per token pair: as many as keep the grid within one
+        // CTA per SM (each block forms its pair's digits)
+        const int pairs = (T + 1) / 2, nmax = (g.n_experts + kRouterBatchExperts - 1) / kRouterBatchExperts;
+        const int nb = std::max(1, std::min(nmax, c->n_sms / pairs));
+        const int eper = (g.n_experts + nb * kRouterBatchExperts - 1) / (nb * kRouterBatchExperts) *
+                         kRouterBatchExperts;
+        const dim3 grid(pairs, (g.n_experts + eper - 1) / eper);
+        k_router_batch<2><<<grid, kRouterBatchThreads, router_batch_smem(2, g.hidden, g.n_experts), s>>>(
             Wr, reinterpret_cast<const __half*>(sc), bias, x, T, g.n_experts, g.hidden, g.top_k,
-            g.renorm, lg, idx, w);
+            g.renorm, eper, lg, c->router_done, idx, w);
         CKL();
         return MOE_OK;
     }

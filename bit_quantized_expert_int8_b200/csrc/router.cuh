@@ -76,7 +76,9 @@ __device__ __forceinline__ void router_select(LP lg, int E, int k, int renorm, i
     }
     int sel[MOE_MAX_TOPK];
     double sel_l[MOE_MAX_TOPK];
-    for (int j = 0; j < k; j++) {
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_TOPK; j++) {
+        if (j >= k) break;
         // lane-local best: largest value, lowest index on ties
         double bv = 0.0;
         int bi = 0x7fffffff;
@@ -95,7 +97,9 @@ __device__ __forceinline__ void router_select(LP lg, int E, int k, int renorm, i
         }
         sel[j] = bi;
         sel_l[j] = bv;
-        if ((bi & 31) == lane) taken[bi >> 5] = true;
+#pragma unroll
+        for (int i = 0; i < kPer; i++)
+            if (bi == lane + 32 * i) taken[i] = true;
     }
     // softmax over all E logits (fp64), then the selected probabilities
     const double m = sel_l[0];
@@ -106,13 +110,18 @@ __device__ __forceinline__ void router_select(LP lg, int E, int k, int renorm, i
         if (ee < E) z += exp(v[i] - m);
     }
     z = warp_sum(z);
-    if (lane == 0) {
-        double p[MOE_MAX_TOPK], zs = 0.0;
-        for (int j = 0; j < k; j++) { p[j] = exp(sel_l[j] - m) / z; zs += p[j]; }
-        for (int j = 0; j < k; j++) {
-            topk_idx[j] = sel[j];
-            topk_w[j] = (float)(renorm ? p[j] / zs : p[j]);
-        }
+    // lane j < k forms p_j; every lane sums them in selection order
+    double lj = 0.0;
+    int ij = 0;
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_TOPK; j++)
+        if (j == lane) { lj = sel_l[j]; ij = sel[j]; }
+    const double pj = lane < k ? exp(lj - m) / z : 0.0;
+    double zs = 0.0;
+    for (int j = 0; j < k; j++) zs += __shfl_sync(0xffffffffu, pj, j);
+    if (lane < k) {
+        topk_idx[lane] = ij;
+        topk_w[lane] = (float)(renorm ? pj / zs : pj);
     }
 }
 
@@ -188,37 +197,47 @@ k_router(const int8_t* __restrict__ W, const __half* __restrict__ scale,
     }
 }
 
-// Steps of many tokens: one CTA per TB tokens and every expert, so a
-// token's digits are formed once and the router matrix is read once per CTA.
-// Each warp takes expert rows two at a time (lanes read consecutive 16-byte
-// chunks of the rows, several chunks in flight) and reduces its TB x NL digit
-// sums across the lanes.  The
-// arithmetic (digits, exact integer row sums, fp64 logits, selection) is that
-// of k_router, so the two kernels choose the same experts with the same
-// weights.  grid ceil(T / TB), block kRouterBatchThreads, dynamic shared
-// memory router_batch_smem(TB, H, E).
+// Steps of many tokens: CTA (token pair, block of eper experts).  The pair's x
+// rows come into shared memory with one pass; their digits are formed there;
+// each warp takes two expert rows of the block (lanes read consecutive
+// 16-byte chunks, several in flight) and reduces its digit sums across the
+// lanes.  The last CTA of a pair (a counter per pair) selects its tokens'
+// experts.  The arithmetic (digits, exact integer row sums, fp64 logits,
+// selection) is that of k_router, so the two kernels choose the same experts
+// with the same weights.  grid (ceil(T / 2), ceil(E / eper)), eper a multiple
+// of 32 (the host picks it so that the grid stays within one wave of CTAs:
+// every CTA forms its pair's digits, so more blocks than SMs cost a second
+// round of that), block kRouterBatchThreads, dynamic shared memory
+// router_batch_smem(2, H, E).
 constexpr int kRouterBatchThreads = 512;
-constexpr int kRouterBatchMinTokens = 128;  // steps from which the batched router runs (measured)
+constexpr int kRouterBatchExperts = 32;     // expert rows per CTA and pass (two per warp)
+constexpr int kRouterBatchMinTokens = 40;   // steps from which the batched router runs (measured)
 __host__ __device__ constexpr size_t router_batch_smem(int TB, int H, int E) {
-    return (size_t)TB * kRouterDigits * H + (size_t)TB * E * sizeof(double);
+    return (size_t)TB * kRouterDigits * H + (size_t)TB * H * 2;
 }
 template <int TB>
 __global__ void __launch_bounds__(kRouterBatchThreads)
 k_router_batch(const int8_t* __restrict__ W, const __half* __restrict__ scale,
                const float* __restrict__ bias, const __half* __restrict__ x, int T, int E, int H,
-               int k, int renorm, double* __restrict__ logits, int32_t* __restrict__ topk_idx,
+               int k, int renorm, int eper, double* __restrict__ logits,
+               int* __restrict__ done_counter, int32_t* __restrict__ topk_idx,
                float* __restrict__ topk_w) {
-    extern __shared__ __align__(16) uint8_t sDig[];   // [TB][kRouterDigits][H], then [TB][E] fp64
-    double* sLg = reinterpret_cast<double*>(sDig + (size_t)TB * kRouterDigits * H);
+    extern __shared__ __align__(16) uint8_t sDig[];   // [TB][kRouterDigits][H], then x [TB][H]
+    __half* sx = reinterpret_cast<__half*>(sDig + (size_t)TB * kRouterDigits * H);
     __shared__ unsigned s_mx[TB];
+    __shared__ int s_last;
     const int t0 = blockIdx.x * TB, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nt = min(TB, T - t0);
     if (tid < TB) s_mx[tid] = 0u;
+    // the pair's rows, one 16-byte load per chunk
+    for (int i = tid; i < nt * (H / 8); i += blockDim.x) {
+        const int t = i / (H / 8), c = i % (H / 8);
+        reinterpret_cast<uint4*>(sx + (size_t)t * H)[c] = reinterpret_cast<const uint4*>(x + (size_t)(t0 + t) * H)[c];
+    }
     __syncthreads();
     for (int t = 0; t < nt; t++) {
-        const __half* xr = x + (size_t)(t0 + t) * H;
         float mx = 0.f;
-        for (int c = tid; c < H; c += blockDim.x) mx = fmaxf(mx, fabsf(__half2float(xr[c])));
+        for (int c = tid; c < H; c += blockDim.x) mx = fmaxf(mx, fabsf(__half2float(sx[(size_t)t * H + c])));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         if (lane == 0) atomicMax(&s_mx[t], __float_as_uint(mx));
@@ -227,17 +246,16 @@ k_router_batch(const int8_t* __restrict__ W, const __half* __restrict__ scale,
     int NL[TB];
 #pragma unroll
     for (int t = 0; t < TB; t++) NL[t] = t < nt ? router_ndigits(__uint_as_float(s_mx[t])) : 0;
-    for (int t = 0; t < nt; t++) {
-        const __half* xr = x + (size_t)(t0 + t) * H;
+    for (int t = 0; t < nt; t++)
         for (int c4 = tid; c4 < H / 4; c4 += blockDim.x)
-            router_digits4(xr, c4, NL[t], sDig + (size_t)t * kRouterDigits * H, H);
-    }
+            router_digits4(sx + (size_t)t * H, c4, NL[t], sDig + (size_t)t * kRouterDigits * H, H);
     __syncthreads();
-    // two expert rows per warp pass, up to 6 chunks of 16 bytes per lane and
-    // row in flight before their dot products
+    // two expert rows per warp, up to 6 chunks of 16 bytes per lane and row in
+    // flight before their dot products
     constexpr int kCh = 6;
-    for (int e0 = 2 * warp; e0 < E; e0 += 2 * (kRouterBatchThreads / 32)) {
-        const bool two = e0 + 1 < E;
+    const int eb = blockIdx.y * eper, ee = min(E, eb + eper);
+    for (int e0 = eb + 2 * warp; e0 < ee; e0 += 2 * (kRouterBatchThreads / 32)) {
+        const bool two = e0 + 1 < ee;
         const int8_t* wr0 = W + (size_t)e0 * H;
         const int8_t* wr1 = W + (size_t)(two ? e0 + 1 : e0) * H;
         int acc[2][TB][kRouterDigits];
@@ -292,19 +310,27 @@ k_router_batch(const int8_t* __restrict__ W, const __half* __restrict__ scale,
 #pragma unroll
                     for (int d = 0; d < kRouterDigits; d++)
                         if (d < NL[t]) S += (long long)warp_sum(acc[r][t][d]) * (1ll << (8 * d));
-                    if (lane == 0) {
-                        const double l = router_logit(S, scale, bias, e);
-                        sLg[t * E + e] = l;
-                        logits[(size_t)(t0 + t) * E + e] = l;
-                    }
+                    if (lane == 0) logits[(size_t)(t0 + t) * E + e] = router_logit(S, scale, bias, e);
                 }
             }
         }
     }
+    // the last CTA of this token pair selects
+    __threadfence();
     __syncthreads();
-    if (warp < nt)
-        router_select(sLg + warp * E, E, k, renorm, lane, topk_idx + (size_t)(t0 + warp) * k,
+    if (tid == 0) {
+        const int prev = atomicAdd(&done_counter[blockIdx.x], 1);
+        s_last = prev == (int)gridDim.y - 1;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (warp < nt) {
+        const volatile double* lg = logits + (size_t)(t0 + warp) * E;
+        router_select(lg, E, k, renorm, lane, topk_idx + (size_t)(t0 + warp) * k,
                       topk_w + (size_t)(t0 + warp) * k);
+    }
+    if (tid == 0) done_counter[blockIdx.x] = 0;       // ready for the next launch
 }
 
 }  // namespace moeq4

@@ -34,11 +34,13 @@ def ctx_for(cfg, T=1):
 
 # ---------------------------------------------------------------- router ----
 
-# T >= 128 runs the batched router (one CTA per two tokens, every expert);
-# 131 tokens leave a CTA with one token.
+# T >= 40 runs the batched router (CTA per token pair and block of experts:
+# 4 blocks of 32 at T = 40 and 64, 2 of 64 at T = 131, one of 128 at T = 256);
+# 131 tokens leave a CTA with one token; TINY's 16 experts fill part of a block.
 @pytest.mark.parametrize("cfg,T,bias", [(TINY, 1, None), (TINY, 7, 1.5), (SMALL, 3, 0.7),
                                         (LAYER, 4, None), (LAYER, 2, 1.5), (TINY, 33, 1.5),
-                                        (LAYER, 64, None), (LAYER, 131, 1.5), (TINY, 128, None)])
+                                        (LAYER, 39, None), (LAYER, 40, 1.5), (LAYER, 64, None),
+                                        (LAYER, 131, 1.5), (TINY, 128, None), (LAYER, 256, 1.5)])
 def test_router_parity(cfg, T, bias):
     L = make_layer(cfg, seed=3, bias_std=bias)
     x = synth.tokens(T, cfg.H, seed=5, device=DEV)
