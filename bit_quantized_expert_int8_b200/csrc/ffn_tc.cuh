@@ -770,17 +770,21 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_cr, const __grid_constant__ CUte
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t bt0 = s_ring + slot * S::kSlot + kTcCodeBytes;
-                    const int ngs = min(2, d.ng - 2 * c);
-                    for (int gi = 0; gi < ngs; gi++) {
-                        const uint32_t dacc = tmem + kTcAccCol + acol + gst * gi;
-                        const uint32_t bt = bt0 + gi * bbytes;
+                    // one descriptor per stage; a K step of 16 elements is 32 bytes (2 in
+                    // the descriptor's address field), a group's half bbytes, a plane brows * 128
+                    const uint64_t bd0 = tc_sdesc_sw128(s_ring + slot * S::kSlot + kTcCodeBytes);
+                    const uint32_t a0 = tmem + 64u * slot, d0 = tmem + kTcAccCol + acol;
+                    const bool two = d.ng - 2 * c > 1;
+#pragma unroll
+                    for (int gi = 0; gi < 2; gi++) {
+                        if (gi == 1 && !two) break;
+                        const uint32_t dacc = d0 + gst * gi;
+                        const uint64_t bdg = bd0 + (uint64_t)((gi * bbytes) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < 4; kk++) {
-                            const uint32_t at = tmem + 64u * slot + 32u * gi + 8u * kk;
-                            tc_mma_ts(dacc, at, tc_sdesc_sw128(bt + 32u * kk), idesc, kk > 0 ? 1u : 0u);
-                            if (DOWN)
-                                tc_mma_ts(dacc, at, tc_sdesc_sw128(bt + brows * 128 + 32u * kk), idesc, 1u);
+                            const uint32_t at = a0 + 32u * gi + 8u * kk;
+                            tc_mma_ts(dacc, at, bdg + 2u * kk, idesc, kk > 0 ? 1u : 0u);
+                            if (DOWN) tc_mma_ts(dacc, at, bdg + (uint64_t)((brows * 128) >> 4) + 2u * kk, idesc, 1u);
                         }
                     }
                     mma_commit(&acc_full[g % kTcAcc]);
