@@ -32,9 +32,10 @@
 //                codes (8 KB, 64-byte swizzle) and two of the B tile (two
 //                64-column halves, 128-byte swizzle; down: both planes) sized
 //                to the tile (16, 32 or 64 rows);
-//   warp 1       MMA issuer: per stage 4 (down: 8) MMAs per group with A in
-//                tensor memory, then one commit that publishes the stage's
-//                accumulators and frees its ring slot and A buffer;
+//   warp 1       MMA issuers (lanes 0 and 1, one scale group each): per
+//                stage 4 (down: 8) MMAs per group with A in tensor memory,
+//                then each lane's commit; the two publish the stage's
+//                accumulators and free its ring slot and A buffer;
 //   warps 2..5   converters: codes -> 16-bit A straight into tensor memory
 //                (tcgen05.st, one row per thread), so A costs no shared-
 //                memory bandwidth;
@@ -666,7 +667,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_cr, const __grid_constant__ CUte
         }
         for (int i = 0; i < kTcAcc; i++) {
             mbar_init(&acc_empty[i], 8);                  // folder warps
-            mbar_init(&acc_full[i], 1);                   // the MMA commit
+            mbar_init(&acc_full[i], 2);                   // the two MMA issuers' commits
         }
         for (int i = 0; i < kTcItemBufs; i++) {
             mbar_init(&ib_full[i], 1);
@@ -742,8 +743,13 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_cr, const __grid_constant__ CUte
             if (ib_last >= 0) mma_drain_wait(&ib_full[ib_last], (uint32_t)((j_last / kTcItemBufs) & 1));
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------- MMA issuer --
-        if (lane == 0) {
+        // --------------------------------------------------- MMA issuers --
+        // Lanes 0 and 1 run the same loop; lane gi issues the MMAs of scale
+        // group gi of every stage (its own accumulator, A columns and B
+        // half), so each MMA instruction of the warp issues two, and each
+        // lane commits its own (the stage barrier takes both arrivals).
+        if (lane < 2) {
+            const int gi = lane;
             uint32_t g = 0, rel = 0, cum_rel = 0;        // stages released, their consumed columns
             uint32_t cumq[kTcAcc];                        // consumed columns after each stage in flight
             TcAccRing ring;
@@ -772,17 +778,13 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tm_cr, const __grid_constant__ CUte
                     tc_fence_after();
                     // one descriptor per stage; a K step of 16 elements is 32 bytes (2 in
                     // the descriptor's address field), a group's half bbytes, a plane brows * 128
-                    const uint64_t bd0 = tc_sdesc_sw128(s_ring + slot * S::kSlot + kTcCodeBytes);
-                    const uint32_t a0 = tmem + 64u * slot, d0 = tmem + kTcAccCol + acol;
-                    const bool two = d.ng - 2 * c > 1;
-#pragma unroll
-                    for (int gi = 0; gi < 2; gi++) {
-                        if (gi == 1 && !two) break;
-                        const uint32_t dacc = d0 + gst * gi;
-                        const uint64_t bdg = bd0 + (uint64_t)((gi * bbytes) >> 4);
+                    const uint64_t bdg = tc_sdesc_sw128(s_ring + slot * S::kSlot + kTcCodeBytes + gi * bbytes);
+                    const uint32_t a0 = tmem + 64u * slot + 32u * gi;
+                    const uint32_t dacc = tmem + kTcAccCol + acol + gst * gi;
+                    if (gi < d.ng - 2 * c) {                  // the stage's group gi exists
 #pragma unroll
                         for (int kk = 0; kk < 4; kk++) {
-                            const uint32_t at = a0 + 32u * gi + 8u * kk;
+                            const uint32_t at = a0 + 8u * kk;
                             tc_mma_ts(dacc, at, bdg + 2u * kk, idesc, kk > 0 ? 1u : 0u);
                             if (DOWN) tc_mma_ts(dacc, at, bdg + (uint64_t)((brows * 128) >> 4) + 2u * kk, idesc, 1u);
                         }
