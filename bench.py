@@ -726,7 +726,7 @@ def run_storage(args):
         os.unlink(path)
 
 
-def bucket_split(counts, T, min_tokens=1, min_step=32):
+def bucket_split(counts, T, min_tokens=1, min_step=2):
     """Experts of one step by the kernel that serves them: `counts` holds the
     pairs routed to each expert.  In steps of at least `min_step` tokens a
     bucket of `min_tokens` or more pairs runs on tcgen05; every other used
@@ -791,10 +791,8 @@ def run_batched(args):
         flop = 2.0 * T * 3 * cfg.H * (cfg.k * cfg.I + cfg.Is)
         if T == 1:
             path = "fused single-token kernel"
-        elif T >= 32:
-            path = "tcgen05 kernels (shared expert and every routed bucket, one persistent launch per FFN half)"
         else:
-            path = "CUDA-core grouped kernels"
+            path = "tcgen05 kernels (shared expert and every routed bucket, one persistent launch per FFN half)"
         lines.append({"tokens": T, "us_per_step": round(us, 2),
                       "us_min_max": [round(min(runs), 2), round(max(runs), 2)],
                       "tokens_per_s": round(T / (us * 1e-6), 1),

@@ -61,7 +61,7 @@ namespace moeq4 {
 constexpr int kMmaRows = 128;                          // M: weight rows per item (TMEM lanes)
 constexpr int kMmaTok = 64;                            // tokens per item at most (N: rounded up to 16)
 constexpr int kMmaDefaultMinTokens = 1;                // bucket size from which a routed expert runs here
-constexpr int kMmaMinStep = 32;                        // tokens in a step before any expert runs here
+constexpr int kMmaMinStep = 2;                         // tokens in a step before any expert runs here (measured)
 constexpr int kTcStageK = 128;                         // K per pipeline stage: two scale groups
 constexpr int kTcCodeBytes = kMmaRows * kTcStageK / 2; // codes of one stage (8 KB)
 constexpr int kTcWarps = 14;

@@ -118,12 +118,12 @@ int moe_set_wait_ns(moe_ctx *ctx, unsigned long long ns);
 /* Multi-token steps with all experts resident group the (token, expert)
  * pairs by expert ("Gemma 4 26B : Comment faire tourner un LLM en 2 Go de
  * RAM", section 04 "Chunked Prefill": one expert applied to many rows).  In a
- * step of at least 32 tokens, an expert whose bucket holds min_tokens or more
+ * step of two or more tokens, an expert whose bucket holds min_tokens or more
  * pairs, and the shared expert once T >= min_tokens, run on the tensor cores
  * (tcgen05; the 4-bit codes and fp16 x are exact operands, h enters as two
  * bf16 planes; fp32 accumulation, one accumulator per 64-column group folded
- * with its scale and bias); the other buckets, and every bucket of a smaller
- * step, run on the CUDA-core grouped kernels.  min_tokens = 0 keeps every
+ * with its scale and bias); the other buckets run on the CUDA-core grouped
+ * kernels (a single token takes the fused layer kernel).  min_tokens = 0 keeps every
  * bucket on the CUDA cores.  The default is 1 where the shape allows the
  * tensor-core kernels (hidden a multiple of 128, the staging buffers within
  * shared memory), else 0.  Host call, no device work.  Returns

@@ -15,8 +15,10 @@ def _bench():
 def test_bucket_split_rules():
     b = _bench()
     counts = [0, 1, 3, 4, 5, 40, 0, 2]
-    # small step: everything on the grouped kernels
-    assert b.bucket_split(counts, T=8) == (0, 6)
+    # a step of one token never reaches these kernels (the fused kernel serves it);
+    # from two tokens every used bucket runs on tcgen05
+    assert b.bucket_split(counts, T=1) == (0, 6)
+    assert b.bucket_split(counts, T=8) == (6, 0)
     # large step: by default every used bucket on tcgen05
     assert b.bucket_split(counts, T=32) == (6, 0)
     # a threshold of 4 pairs leaves the smaller buckets on the grouped kernels

@@ -79,14 +79,16 @@ def test_ep_dispatch_rejects_bad_shapes():
     assert e.value.code == moeq4.MOE_ERR_UNSUPPORTED_SHAPE
 
 
-@pytest.mark.parametrize("R", [20, 100])
-def test_ffn_rows_matches_oracle(R):
-    """R = 20 rows run on the CUDA-core grouped kernels, R = 100 on tcgen05;
-    16 local experts with uneven row counts (some none).  A context of
-    ceil(2 R / (k + 1)) tokens is the smallest that holds R rows."""
+@pytest.mark.parametrize("R,tau", [(20, 0), (20, 1), (100, 1)])
+def test_ffn_rows_matches_oracle(R, tau):
+    """Rows on the CUDA-core grouped kernels (tensor-core threshold 0) and on
+    tcgen05 (threshold 1); 16 local experts with uneven row counts (some
+    none).  A context of ceil(2 R / (k + 1)) tokens is the smallest that holds
+    R rows."""
     cfg = LAYER
     L = make_layer(cfg, seed=51)
     ctx = moeq4.Context(cfg, -(-2 * R // (cfg.k + 1)))
+    moeq4.moe_set_mma_min_tokens(ctx, tau)
     n_local = 16
     g = torch.Generator().manual_seed(R)
     rows_e = torch.randint(0, n_local - 3, (R,), generator=g, dtype=torch.int32).to(DEV)

@@ -1,13 +1,12 @@
 """Tensor-core (tcgen05) buckets of the multi-token path against the oracle.
 
-Multi-token steps group the (token, expert) pairs by expert; in a step of at
-least 32 tokens a bucket of at least the configured size (and the shared
+Multi-token steps group the (token, expert) pairs by expert; in a step of two
+or more tokens a bucket of at least the configured size (and the shared
 expert once T reaches it) runs on the tensor cores.  These tests force every
 bucket of such steps onto that path (threshold 1, buckets of one pair up),
 concentrate whole steps on eight experts (buckets of 130 pairs: tiles of 64,
 64 and a ragged 2), and compare each token with the oracle and with the
-CUDA-core path.  A step of 8 tokens stays on the CUDA cores whatever the
-threshold.
+CUDA-core path (threshold 0).
 """
 import numpy as np
 import pytest
@@ -82,7 +81,8 @@ def test_mma_every_bucket_tiny():
 
 @pytest.mark.parametrize("T,sample", [(8, tuple(range(8))), (200, (0, 63, 64, 130, 199))])
 def test_mma_layer_small_buckets(T, sample):
-    """Layer shape, threshold 1: T = 8 (below the step size: CUDA cores) and
+    """Layer shape, threshold 1: T = 8 (buckets of one or two pairs, each a
+    16-row tile, and the shared expert's 8 tokens on the tensor cores) and
     T = 200 (every bucket, about a dozen pairs each, on the tensor cores; the
     shared expert in tiles of 64, 64, 64 and 8)."""
     cfg = LAYER

@@ -214,12 +214,14 @@ def test_layer_resident_parity(cfg, T, bias):
                                                (LAYER, 2, None, (0, 1)),
                                                (SMALL, 33, 0.7, tuple(range(33)))])
 def test_layer_grouped_multi_token(cfg, T, bias, sample):
-    """T > 1 runs the grouped path (each expert read once for all of its
-    tokens, tokens in passes of 4, ragged last pass); sampled tokens against
-    the oracle, and the same step split into single-token calls."""
+    """T > 1 on the CUDA-core grouped path (tensor-core threshold 0: each
+    expert read once for all of its tokens, tokens in passes of 4, ragged last
+    pass); sampled tokens against the oracle, and the same step split into
+    single-token calls."""
     L = make_layer(cfg, seed=4, bias_std=bias)
     x = synth.tokens(T, cfg.H, seed=14, device=DEV)
     ctx = ctx_for(cfg, T)
+    moeq4.moe_set_mma_min_tokens(ctx, 0)
     lay = moeq4.Layer.from_dict(L)
     y = torch.empty((T, cfg.H), device=DEV)
     idx = torch.empty((T, cfg.k), dtype=torch.int32, device=DEV)
