@@ -252,14 +252,16 @@ __device__ __forceinline__ int tc_col_pos(int c) {
 // expert), r = T + i is the token of the i-th pair in bucket order
 // (list[i] / k).  Copies the fp16 row into xs[r] with each 8 columns in the
 // tensor-core order and writes its 64-column group sums gsum[r][g] (fp32,
-// row stride gs_stride).  One warp per 256 columns; grid y strides over the
-// rows.
+// row stride gs_stride).  n_pairs (device, or null for all T k): the pairs
+// the list holds, when a grouping selected only some of them.  One warp per
+// 256 columns; grid y strides over the rows.
 __global__ void k_gather_x(const __half* __restrict__ x, int H, int T, int k, int rows,
                            const int* __restrict__ list, __half* __restrict__ xs,
-                           float* __restrict__ gsum, int gs_stride) {
+                           float* __restrict__ gsum, int gs_stride, const int* __restrict__ n_pairs) {
     const int lane = threadIdx.x & 31;
     const int c0 = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 256 + 8 * lane;
     if (c0 - 8 * lane >= H) return;                       // whole warp past the row end
+    if (n_pairs) rows = min(rows, T + *n_pairs);
     for (int r = blockIdx.y; r < rows; r += gridDim.y) {
         const int tok = r < T ? r : list[r - T] / k;
         float s = 0.f;

@@ -608,7 +608,8 @@ extern "C" int moe_combine(moe_ctx* c, const float* y_routed, const float* y_sha
 }
 
 static int ffn_grouped(moe_ctx* c, const uint8_t* ex, int E, const uint8_t* sh, const __half* xin,
-                       const int32_t* idx, int T, int k, cudaStream_t s);
+                       const int32_t* idx, int T, int k, cudaStream_t s, const int32_t* sel = nullptr,
+                       int sel_val = 0, bool routed = true);
 
 extern "C" int moe_ep_dispatch(moe_ctx* c, const int32_t* topk_idx, int T, int n_ranks,
                                const moe_half* x, moe_half* send_x, int32_t* send_expert,
@@ -703,9 +704,12 @@ extern "C" int moe_cache_lookup_lfu(moe_ctx* c, MoeLfuTable* table, const int32_
 // Multi-token FFNs of all experts resident (T >= 1 tokens, k pairs each,
 // pair q = t * k + j choosing idx[q] < E): outputs in c->y_pairs, row t for
 // the shared expert (when sh is given) and row T + q for pair q.  Each expert
-// is read once for all of its tokens.
+// is read once for all of its tokens.  sel (device, optional): only the pairs
+// with sel[q] == sel_val (a batch of cache slots); routed = false: the shared
+// expert alone.
 static int ffn_grouped(moe_ctx* c, const uint8_t* ex, int E, const uint8_t* sh, const __half* xin,
-                       const int32_t* idx, int T, int k, cudaStream_t s) {
+                       const int32_t* idx, int T, int k, cudaStream_t s, const int32_t* sel,
+                       int sel_val, bool routed) {
     {
         const MoeConfig& g = c->cfg;
         const int H = g.hidden;
@@ -722,14 +726,16 @@ static int ffn_grouped(moe_ctx* c, const uint8_t* ex, int E, const uint8_t* sh, 
         const int cap = tc ? tau : 0x7fffffff;
         const int P = T * (k + 1), hs = c->maxI;
         __nv_bfloat16 *hh = c->h_pl, *hl = c->h_pl + (size_t)P * hs;
-        k_group_pairs<<<1, 1024, 0, s>>>(idx, T * k, E, c->e_off, c->plist);
+        if (!routed) sel_val = -1;                    // no pair is grouped
+        k_group_pairs<<<1, 1024, 0, s>>>(idx, T * k, E, c->e_off, c->plist, routed ? sel : idx, sel_val);
         CKL();
         CUtensorMap m_cgr, m_cgs, m_cdr, m_cds, m_x[3], m_h[3];
         TcArgs ta{};
         if (tc) {
             // x rows in bucket order (tokens first) with their group sums; this call's tensor maps
             k_gather_x<<<dim3((H + 2047) / 2048, P < 65535 ? P : 65535), 256, 0, s>>>(
-                xin, H, T, k, P, c->plist, c->xs, c->xg_sum, c->xg_stride);
+                xin, H, T, k, P, c->plist, c->xs, c->xg_sum, c->xg_stride,
+                (sel || !routed) ? c->e_off + E : nullptr);
             CKL();
             const BlobLayout Lr(H, I), Ls(H, Is);
             const size_t sb = Ls.bytes;
@@ -742,14 +748,14 @@ static int ffn_grouped(moe_ctx* c, const uint8_t* ex, int E, const uint8_t* sh, 
                       encode_rows(&m_h[b], hh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hs, P, 2, 16 << b);
             if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed");
             ta.H = H; ta.T = T; ta.k = k; ta.E = E; ta.gelu = g.gelu;
-            ta.Ir = I; ta.Is = Is; ta.min_tok = tau; ta.do_shared = tc_shared ? 1 : 0;
+            ta.Ir = I; ta.Is = Is; ta.min_tok = routed ? tau : 0x7fffffff; ta.do_shared = tc_shared ? 1 : 0;
             ta.e_off = c->e_off; ta.list = c->plist;
             ta.h_hi = hh; ta.h_lo = hl; ta.h_sum = c->h_sum; ta.hs = hs; ta.hsum_stride = c->hsum_stride;
             ta.y_pairs = c->y_pairs; ta.status = c->status;
         }
         const int chunks = (T + kGrpChunk - 1) / kGrpChunk;
         // with a threshold of one pair every routed bucket is on the tensor cores
-        const bool grp_routed = !(tc && tau <= 1);
+        const bool grp_routed = routed && !(tc && tau <= 1);
         if (grp_routed) {
             k_gateup_grouped<false><<<dim3(I / 16, E), kGrpThreads, grouped_smem_gu(H), s>>>(
                 ex, stride, sh, H, I, xin, T, k, c->e_off, c->plist, cap, g.gelu, c->h_ws, c->maxI);
@@ -953,7 +959,7 @@ static int layer_streaming_fused(moe_ctx* c, const MoeLayer* L, __half* x, const
 static int layer_streaming_chunk(moe_ctx* c, const MoeLayer* L, __half* x, int T, const MoeLayerOut* o,
                                  int flags, cudaStream_t s, cudaStream_t cs) {
     const MoeConfig& g = c->cfg;
-    const int k = g.top_k, H = g.hidden, I = g.inter, Is = g.inter_shared, E = g.n_experts;
+    const int k = g.top_k, H = g.hidden, I = g.inter, E = g.n_experts;
     const bool dev_fill = (flags & MOE_DEVICE_FILL) != 0;
     const size_t stride = BlobLayout(H, I).bytes;
     const __half* xin = x;
@@ -980,18 +986,13 @@ static int layer_streaming_chunk(moe_ctx* c, const MoeLayer* L, __half* x, int T
     k_lfu_chunk<<<1, 32, 0, s>>>(L->lfu, idx, T, k, E, slot_of, c->batch_of, c->plan_dev, c->status);
     CKL();
     CK(cudaEventRecord(c->ev_lookup, s));
-    // the shared expert for every token of the chunk, while the host reads
-    // the plan and the first batch's misses are filled
+    // the shared expert for every token of the chunk (the kernels of a
+    // resident step: tensor cores from two tokens), while the host reads the
+    // plan and the first batch's misses are filled
     const uint8_t* sh = static_cast<const uint8_t*>(L->shared_blob);
     uint8_t* slots = static_cast<uint8_t*>(L->slots);
     const uint8_t* store = static_cast<const uint8_t*>(L->host_store);
-    const int chunks = (T + kGrpChunk - 1) / kGrpChunk;
-    k_gateup_grouped<true><<<dim3(Is / 16, 1, chunks), kGrpThreads, grouped_smem_gu(H), s>>>(
-        slots, stride, sh, H, Is, xin, T, k, c->e_off, c->plist, 0x7fffffff, g.gelu, c->h_ws, c->maxI);
-    CKL();
-    k_down_grouped<true><<<dim3(H / 16, 1, chunks), kGrpThreads, grouped_smem_dn(Is), s>>>(
-        slots, stride, sh, H, Is, T, c->e_off, c->plist, 0x7fffffff, c->h_ws, c->maxI, c->y_pairs);
-    CKL();
+    TRY(ffn_grouped(c, slots, MOE_MAX_SLOTS, sh, xin, slot_of, T, k, s, nullptr, 0, false));
     CK(cudaEventSynchronize(c->ev_lookup));
     const int max_b = E + 1;
     const int nb = *(volatile int32_t*)c->plan_host;
@@ -1036,15 +1037,9 @@ static int layer_streaming_chunk(moe_ctx* c, const MoeLayer* L, __half* x, int T
             CK(cudaEventRecord(c->ev_copy, cs));
             CK(cudaStreamWaitEvent(s, c->ev_copy, 0));
         }
-        // the batch's routed pairs grouped by cache slot
-        k_group_pairs<<<1, 1024, 0, s>>>(slot_of, T * k, MOE_MAX_SLOTS, c->e_off, c->plist, c->batch_of, b);
-        CKL();
-        k_gateup_grouped<false><<<dim3(I / 16, MOE_MAX_SLOTS), kGrpThreads, grouped_smem_gu(H), s>>>(
-            slots, stride, sh, H, I, xin, T, k, c->e_off, c->plist, 0x7fffffff, g.gelu, c->h_ws, c->maxI);
-        CKL();
-        k_down_grouped<false><<<dim3(H / 16, MOE_MAX_SLOTS), kGrpThreads, grouped_smem_dn(I), s>>>(
-            slots, stride, sh, H, I, T, c->e_off, c->plist, 0x7fffffff, c->h_ws, c->maxI, c->y_pairs);
-        CKL();
+        // the batch's routed pairs grouped by cache slot, through the kernels
+        // of a resident step (each expert's bucket is whole within its batch)
+        TRY(ffn_grouped(c, slots, MOE_MAX_SLOTS, nullptr, xin, slot_of, T, k, s, c->batch_of, b, true));
         CK(cudaEventRecord(c->ev_ffn, s));
     }
     TRY(launch_combine(c, c->y_pairs + (size_t)T * H, c->y_pairs, w, T, o->y,

@@ -5,15 +5,16 @@ cache ("Gemma 4 26B : Comment faire tourner un LLM en 2 Go de RAM", section
 chunk that uses it).
 
 The chunk is one cache lookup: its distinct experts are served in batches
-that fit the slots, each expert copied at most once, and the grouped kernels
-serve each batch's (token, choice) pairs from the slots.
+that fit the slots, each expert copied at most once, and the kernels of a
+resident multi-token step (tensor cores, or the CUDA-core grouped kernels at
+threshold 0) serve each batch's (token, choice) pairs from the slots.
 
 Checks at the layer shape (hidden 2816, 128 experts, top-8, 16 slots, router
 bias N(0, 1.5)), two layers, a 96-token prompt with RMSNorm and the fp16
 residual, both fill modes:
 - streaming output equals the resident batched output bit for bit, y and the
-  residual (both on the CUDA-core grouped kernels: the tensor-core threshold
-  is set to 0 on the resident side, the streaming side never uses them);
+  residual, with both on the tensor cores (default threshold) and both on
+  the CUDA-core grouped kernels (threshold 0);
 - the slot of every (token, choice), each layer's table and its hit and miss
   totals equal the oracle's chunk model run on the GPU's routing, and no
   expert is copied twice in a chunk;
@@ -71,13 +72,15 @@ def _oracle_state(c):
     return (c.expert.tolist(), c.count.tolist(), c.seq.tolist(), int(c.hits[0]), int(c.misses[0]), 1)
 
 
-@pytest.mark.parametrize("fill", ["host", "device"])
-def test_chunk_layer_shape_resident_oracle_and_cache(fill):
+@pytest.mark.parametrize("fill,tau", [("host", None), ("device", None), ("host", 0)])
+def test_chunk_layer_shape_resident_oracle_and_cache(fill, tau):
     cfg, T, n_layers = LAYER, 96, 2
     stack = _stack(cfg, n_layers, seed=17, bias_std=1.5)
     flags = moeq4.MOE_PRENORM | (moeq4.MOE_DEVICE_FILL if fill == "device" else 0)
     ctx_st, ctx_rs = moeq4.Context(cfg, T), moeq4.Context(cfg, T)
-    moeq4.moe_set_mma_min_tokens(ctx_rs, 0)               # resident side on the grouped kernels too
+    if tau is not None:                                   # both sides on the grouped kernels
+        moeq4.moe_set_mma_min_tokens(ctx_st, tau)
+        moeq4.moe_set_mma_min_tokens(ctx_rs, tau)
     cs = torch.cuda.Stream()
     caches = [oracle.LfuCache(cfg.S) for _ in stack]
     for s in stack:
@@ -123,7 +126,6 @@ def test_chunks_of_several_sizes_tiny(fill):
     s = stack[0]
     flags = moeq4.MOE_PRENORM | (moeq4.MOE_DEVICE_FILL if fill == "device" else 0)
     ctx_st, ctx_rs = moeq4.Context(cfg, 40), moeq4.Context(cfg, 40)
-    moeq4.moe_set_mma_min_tokens(ctx_rs, 0)
     cs = torch.cuda.Stream()
     moeq4.moe_lfu_init(ctx_st, s["table"], cfg.S)
     cache = oracle.LfuCache(cfg.S)
