@@ -79,6 +79,21 @@ def test_mma_every_bucket_tiny():
         assert_y_close(y_tc[t], y_cc[t].astype(np.float64), f"tensor vs CUDA cores, token {t}")
 
 
+@pytest.mark.parametrize("cfg,T", [(LAYER, 2), (LAYER, 3), (TINY, 2), (TINY, 5)])
+def test_mma_smallest_steps_match_oracle_and_cuda_cores(cfg, T):
+    """The smallest multi-token steps on the tensor cores: one-pair buckets
+    (16-row tiles holding one or two tokens) and a shared expert of T tokens;
+    every token against the oracle and against the CUDA-core path."""
+    L = make_layer(cfg, seed=27 + T, bias_std=1.5)
+    x = synth.tokens(T, cfg.H, seed=28 + T, device=DEV)
+    y_tc, idx_tc = _run(cfg, L, x, T, 1)
+    y_cc, idx_cc = _run(cfg, L, x, T, 0)
+    np.testing.assert_array_equal(idx_tc, idx_cc)
+    _check_tokens(cfg, L, x, y_tc, idx_tc, range(T))
+    for t in range(T):
+        assert_y_close(y_tc[t], y_cc[t].astype(np.float64), f"tensor vs CUDA cores, token {t}")
+
+
 @pytest.mark.parametrize("T,sample", [(8, tuple(range(8))), (200, (0, 63, 64, 130, 199))])
 def test_mma_layer_small_buckets(T, sample):
     """Layer shape, threshold 1: T = 8 (buckets of one or two pairs, each a
