@@ -662,6 +662,25 @@ extern "C" int moe_ffn_rows(moe_ctx* c, const void* experts, int n_experts, cons
     return MOE_OK;
 }
 
+extern "C" int moe_shared_ffn(moe_ctx* c, const void* shared_blob, const moe_half* x, int T, float* y,
+                              moe_stream_t stream) {
+    if (!c || !shared_blob || !x || !y) return fail(MOE_ERR_INVALID_ARG, "moe_shared_ffn: NULL argument");
+    if (T < 1 || T > c->maxT) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T=%d outside 1..%d", T, c->maxT);
+    if (!c->grouped_ok)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_shared_ffn needs the grouped kernels for this shape");
+    if (!aligned16(shared_blob) || !aligned16(x) || !aligned16(y))
+        return fail(MOE_ERR_ALIGNMENT, "moe_shared_ffn: pointers must be 16-byte aligned");
+    const MoeConfig& g = c->cfg;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint8_t* sh = static_cast<const uint8_t*>(shared_blob);
+    // the shared expert alone: no pair is grouped (the routing argument is
+    // only read, never used)
+    TRY(ffn_grouped(c, sh, 1, sh, reinterpret_cast<const __half*>(x), c->idx, T, g.top_k, s, nullptr, 0,
+                    false));
+    CK(cudaMemcpyAsync(y, c->y_pairs, (size_t)T * g.hidden * sizeof(float), cudaMemcpyDeviceToDevice, s));
+    return MOE_OK;
+}
+
 extern "C" int moe_ep_unpermute(moe_ctx* c, const float* y_sorted, const int32_t* send_order, int n,
                                 float* y_pairs, moe_stream_t stream) {
     if (!c || !y_sorted || !send_order || !y_pairs)

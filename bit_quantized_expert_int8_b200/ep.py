@@ -13,7 +13,7 @@ rank's T tokens:
    the grouped / tensor-core kernels, one expert read once for all its rows);
 5. all-to-all of the output rows back to the ranks they came from;
 6. rows back in pair order (``moe_ep_unpermute``), the shared expert
-   (``moe_expert_ffn_q4``) and the fixed-order combine (``moe_combine``).
+   (``moe_shared_ffn``) and the fixed-order combine (``moe_combine``).
 
 The pages run one process on one machine (the per-expert FFN of their
 pipeline, step 2-3 of section 04 of "Gemma 4 26B : Comment faire tourner un
@@ -114,9 +114,7 @@ class CudaEpBackend:
 
     def shared(self, x, T):
         y = torch.empty((T, self.H), dtype=torch.float32, device=self.device)
-        pairs = moeq4.make_pairs([(self.shared_blob.data_ptr(), self.cfg.Is, t) for t in range(T)],
-                                 self.device)
-        moeq4.moe_expert_ffn_q4(self.ctx, pairs, T, x, T, y)
+        moeq4.moe_shared_ffn(self.ctx, self.shared_blob, x, T, y)
         return y
 
     def combine(self, y_pairs, y_sh, w, T):

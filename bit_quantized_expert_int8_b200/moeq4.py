@@ -31,7 +31,7 @@ MOE_MAX_SLOTS = 32
 EXPORTS = ("moe_ctx_create", "moe_ctx_destroy", "moe_ctx_check", "moe_ctx_trace", "moe_ctx_info",
            "moe_last_error", "moe_blob_bytes",
            "moe_router_topk", "moe_expert_ffn_q4", "moe_combine", "moe_lfu_init",
-           "moe_ep_dispatch", "moe_ffn_rows", "moe_ep_unpermute",
+           "moe_ep_dispatch", "moe_ffn_rows", "moe_shared_ffn", "moe_ep_unpermute",
            "moe_cache_lookup_lfu", "moe_layer_decode", "moe_stack_decode",
            "moe_router_topk_noalloc", "moe_set_mma_min_tokens", "moe_set_wait_ns",
            "moe_store_stride", "moe_store_open", "moe_store_close", "moe_store_read",
@@ -104,6 +104,7 @@ def load() -> ctypes.CDLL:
         "moe_combine": ([P, P, P, P, i32, P, P, P], i32),
         "moe_ep_dispatch": ([P, P, i32, i32, P, P, P, P, P, P], i32),
         "moe_ffn_rows": ([P, P, i32, P, i32, P, P, P], i32),
+        "moe_shared_ffn": ([P, P, P, i32, P, P], i32),
         "moe_ep_unpermute": ([P, P, P, i32, P, P], i32),
         "moe_lfu_init": ([P, P, i32, P], i32),
         "moe_cache_lookup_lfu": ([P, P, P, i32, P, P, P, P], i32),
@@ -262,6 +263,10 @@ def moe_ep_dispatch(ctx, topk_idx, T, n_ranks, x, send_x, send_expert, send_orde
 def moe_ffn_rows(ctx, experts, n_experts, expert_of_row, R, x_rows, y_rows, stream=None):
     _check(load().moe_ffn_rows(ctx.handle, _ptr(experts), n_experts, _ptr(expert_of_row), R,
                                _ptr(x_rows), _ptr(y_rows), _stream(stream)))
+
+
+def moe_shared_ffn(ctx, shared_blob, x, T, y, stream=None):
+    _check(load().moe_shared_ffn(ctx.handle, _ptr(shared_blob), _ptr(x), T, _ptr(y), _stream(stream)))
 
 
 def moe_ep_unpermute(ctx, y_sorted, send_order, n, y_pairs, stream=None):

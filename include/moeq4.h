@@ -281,6 +281,17 @@ int moe_ep_dispatch(moe_ctx *ctx, const int32_t *topk_idx, int T, int n_ranks,
 int moe_ffn_rows(moe_ctx *ctx, const void *experts, int n_experts, const int32_t *expert_of_row,
                  int R, const moe_half *x_rows, float *y_rows, moe_stream_t stream);
 
+/* moe_shared_ffn: the shared expert, which every token runs next to its
+ * routed experts ([LH] 04 pipeline: the shared expert is always computed;
+ * [RM] "L'affirmation des 2 Go ..."), applied to T token rows:
+ * y[t] = down(GELU(gate x_t) * up x_t) with the shared blob (device, layout
+ * of moe_blob_bytes(H, inter_shared)), through the kernels of a resident
+ * multi-token step (the tensor cores from two tokens, else the CUDA-core
+ * grouped kernels).  x device fp16 [T][H], y device fp32 [T][H]; T must be
+ * 1..max_tokens. */
+int moe_shared_ffn(moe_ctx *ctx, const void *shared_blob, const moe_half *x, int T, float *y,
+                   moe_stream_t stream);
+
 /* moe_ep_unpermute: rows returned in send order back to pair order,
  * y_pairs[send_order[p]] = y_sorted[p] for p < n (device fp32 rows of H). */
 int moe_ep_unpermute(moe_ctx *ctx, const float *y_sorted, const int32_t *send_order, int n,

@@ -105,6 +105,25 @@ def test_ffn_rows_matches_oracle(R, tau):
         assert_y_close(yc[r], ref, f"row {r}")
 
 
+@pytest.mark.parametrize("T", [1, 2, 37])
+def test_shared_ffn_matches_oracle(T):
+    """moe_shared_ffn: T = 1 on the CUDA-core grouped kernels, T = 2 and 37 on
+    tcgen05 (tiles of 16 and 64 rows), every row against the oracle."""
+    cfg = LAYER
+    L = make_layer(cfg, seed=56)
+    ctx = moeq4.Context(cfg, T)
+    x = synth.tokens(T, cfg.H, seed=57 + T, device=DEV)
+    y = torch.empty((T, cfg.H), device=DEV)
+    moeq4.moe_shared_ffn(ctx, L["shared"], x, T, y)
+    moeq4.moe_ctx_check(ctx)
+    xs = np_of(x).view(np.float16).astype(np.float64)
+    sh = np_of(L["shared"])
+    yc = y.cpu().numpy()
+    for t in range(T):
+        ref = oracle.expert_ffn(sh, cfg.H, cfg.Is, xs[t], cfg.gelu)[0]
+        assert_y_close(yc[t], ref, f"row {t}")
+
+
 def test_ep_layer_emulated_four_ranks():
     """Four ranks of 32 experts each on one GPU, 40, 8, 64 and 1 tokens: every
     rank's device steps in turn, rows moved between them on the host in the
