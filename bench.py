@@ -54,7 +54,7 @@ def parse():
     p.add_argument("--store-dir", default=tempfile.gettempdir(), help="directory of the expert file")
     p.add_argument("--store-layers", type=int, default=8, help="layers in the expert file")
     p.add_argument("--store-threads", type=int, default=16, help="pread threads")
-    p.add_argument("--workload", choices=("stack", "streaming", "batched", "prefill", "storage"),
+    p.add_argument("--workload", choices=("stack", "streaming", "batched", "prefill", "storage", "direct"),
                    default="stack",
                    help="stack (default, the headline line), streaming (experts in pinned host "
                         "memory behind the LFU cache), batched (one layer, T tokens per step) or "
@@ -815,6 +815,59 @@ def run_batched(args):
                       "tensor_peak_kind": tkind, "mma_min_tokens": 1, "sweep": lines}), flush=True)
 
 
+def run_direct(args):
+    """The granular expert-FFN entry point (moe_expert_ffn_q4, direct
+    per-pair kernels) on one token's pairs of the stack configuration: the
+    shared expert and 8 routed experts, each blob read once per call; 8
+    weight copies rotated so no call finds its blobs in L2."""
+    import torch
+
+    from bit_quantized_expert_int8_b200 import moeq4, synth
+    from bit_quantized_expert_int8_b200.config import LAYER
+    cfg = LAYER
+    dev = torch.device("cuda", 0)
+    moeq4.load()
+    hbm, kind = peaks()
+    copies = [synth.layer_weights(cfg, SEED, l, dev) for l in range(8)]
+    nb, nbs = synth.blob_bytes(cfg.H, cfg.I), synth.blob_bytes(cfg.H, cfg.Is)
+    ctx = moeq4.Context(cfg, 1)
+    x = synth.tokens(1, cfg.H, SEED + 3, dev)
+    y = torch.empty((cfg.k + 1, cfg.H), dtype=torch.float32, device=dev)
+    pair_sets = []
+    for d in copies:
+        base = d["experts"].data_ptr()
+        ent = [(d["shared"].data_ptr(), cfg.Is, 0)]
+        ent += [(base + e * 16 * nb, cfg.I, 0) for e in range(cfg.k)]     # experts 0, 16, ..., 112
+        pair_sets.append(moeq4.make_pairs(ent, dev))
+    for p in pair_sets:                                                     # warm up
+        moeq4.moe_expert_ffn_q4(ctx, p, cfg.k + 1, x, 1, y)
+    reps = 200
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(0)
+    clocks.start()
+    runs = []
+    for _ in range(REPEATS):
+        torch.cuda.synchronize()
+        e0.record()
+        for r in range(reps):
+            moeq4.moe_expert_ffn_q4(ctx, pair_sets[r % len(pair_sets)], cfg.k + 1, x, 1, y)
+        e1.record()
+        torch.cuda.synchronize()
+        runs.append(e0.elapsed_time(e1) * 1000.0 / reps)
+    clk = clocks.stop()
+    moeq4.moe_ctx_check(ctx)
+    us = statistics.median(runs)
+    algo = cfg.k * nb + nbs
+    print(json.dumps({"metric": METRIC, "workload": "direct: moe_expert_ffn_q4, one token, "
+                                                    "shared + 8 routed experts",
+                      "unit": "us per call", "value": round(us, 2),
+                      "us_min_max": [round(min(runs), 2), round(max(runs), 2)],
+                      "timing": f"median of {REPEATS} runs of {reps} calls", "clocks": clk,
+                      "algorithmic_bytes": algo, "achieved_gbs": round(algo / (us * 1e-6) / 1e9, 1),
+                      "frac_of_hbm": round(algo / (us * 1e-6) / 1e9 / hbm, 4), "peak_kind": kind,
+                      "kernels": "k_ffn_gateup_simple + k_ffn_down_simple"}), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -827,6 +880,8 @@ def main():
         run_prefill(args)
     elif args.workload == "storage":
         run_storage(args)
+    elif args.workload == "direct":
+        run_direct(args)
     else:
         run_ours(args)
 
